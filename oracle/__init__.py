@@ -1,0 +1,2 @@
+"""Float64 CPU oracle (test infrastructure only; the library never imports it)."""
+from .fva_oracle import *  # noqa: F401,F403
