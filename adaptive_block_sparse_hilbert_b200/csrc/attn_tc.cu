@@ -1,0 +1,432 @@
+// Block-sparse (and dense) flash-style forward attention on sm_100a tensor cores.
+//
+// Method: aixai.ru FVAttn blog, sparse-attention section -- attention is computed only
+// over the key blocks the router kept for a query block; the dense case (every block
+// kept) is the FlashAttention-style baseline the pages compare against.
+//
+// Design (B200):
+//   * One CTA per tile = two Hilbert-adjacent query blocks (128 query rows) of one
+//     (b, h). It walks the union of the two rows' kept key-block lists; each list entry
+//     carries which of the two query blocks keeps it, and the other half's scores are
+//     masked to -inf. A 128-row tile never costs more tensor time than two 64-row
+//     (M=64, half-rate) tiles, and Hilbert-adjacent blocks share most of their lists.
+//   * Warp roles: warp 4 issues TMA tile loads (Q once, then K and V blocks of 64 keys
+//     into a ring of stages), warp 5 issues tcgen05.mma (one thread), warps 0-3 own one
+//     query row per thread (TMEM lane) for the online softmax and the epilogue.
+//   * S = Q K^T (M=128, N=64, K=d, bf16 -> fp32) goes to one of two TMEM buffers; the
+//     softmax warps read it, write P back over it as packed bf16 and the MMA warp
+//     issues O += P V with P taken straight from TMEM (A operand) and V from shared
+//     memory (B operand, MN-major). O stays in TMEM until the epilogue.
+//   * O is rescaled only when a row maximum grows by more than 2^8 (log2 units), so
+//     the exponentials stay <= 256 and the TMEM read-modify-write of O is rare.
+//   * Two CTAs per SM (<= 256 TMEM columns and ~97 KB smem each): while one CTA runs
+//     its softmax, the other keeps the tensor core busy.
+//   * Tiles are launched in the order of the work list (longest first); the hardware
+//     block scheduler hands each free CTA slot the next tile, i.e. greedy list
+//     scheduling.
+//   * Every mbarrier wait is bounded (~2 s); on expiry the CTA reports
+//     FVA_DEVERR_TIMEOUT, drains its own TMA loads and MMAs, frees TMEM and exits.
+#include <math.h>
+
+#include "fva_internal.cuh"
+
+namespace fva {
+
+constexpr int kAttnThreads = 192;
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 64;   // keys per step (one key block)
+constexpr uint32_t kTmemCols = 256;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Bounded wait taken by a whole warp: the result is the same on every lane, so the
+// warp stays converged for the .sync.aligned TMEM instructions that follow.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const bool ok = mbar_wait(bar, parity, abort, kWaitLimitNs);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int D>
+struct AttnCfg {
+  static constexpr int kChunks = D / 64;                    // 128-byte swizzle rows per d
+  static constexpr int kStages = (D == 128) ? 2 : 4;
+  static constexpr int kQBytes = kChunks * kBM * 128;        // 128 rows x 128 B per chunk
+  static constexpr int kKVBytes = kChunks * kBN * 128;       // 64 rows x 128 B per chunk
+  static constexpr int kSmemData = kQBytes + 2 * kStages * kKVBytes;
+  static constexpr uint32_t kOCol = 128;                     // O columns [128, 128 + D)
+};
+
+template <int D>
+struct __align__(8) AttnBars {
+  uint64_t q_full;
+  uint64_t k_full[AttnCfg<D>::kStages];
+  uint64_t k_empty[AttnCfg<D>::kStages];
+  uint64_t v_full[AttnCfg<D>::kStages];
+  uint64_t v_empty[AttnCfg<D>::kStages];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t pv_done;
+  uint64_t o_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D>
+constexpr size_t attn_smem_bytes() {
+  return 1024 /*alignment slack*/ + AttnCfg<D>::kSmemData + sizeof(AttnBars<D>);
+}
+
+template <int D, bool DENSE>
+__global__ void __launch_bounds__(kAttnThreads, 2)
+    attn_bf16_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                     const __grid_constant__ CUtensorMap tmv, __nv_bfloat16* __restrict__ out,
+                     const int32_t* __restrict__ tile_ptr, const int32_t* __restrict__ tile_col,
+                     const int32_t* __restrict__ worklist, int N, int nB, int nPairs, float scale_log2,
+                     int32_t* dev_status) {
+  using Cfg = AttnCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + Cfg::kQBytes;
+  uint8_t* sV = sK + Cfg::kStages * Cfg::kKVBytes;
+  AttnBars<D>& bar = *reinterpret_cast<AttnBars<D>*>(smem + Cfg::kSmemData);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = DENSE ? static_cast<int>(blockIdx.x) : worklist[blockIdx.x];
+  const int bh = tile / nPairs;
+  const int t = tile - bh * nPairs;
+  int n_iter, list_base;
+  if (DENSE) {
+    n_iter = nB;
+    list_base = 0;
+  } else {
+    list_base = tile_ptr[tile];
+    n_iter = tile_ptr[tile + 1] - list_base;
+  }
+
+  if (threadIdx.x == 128) {
+    tma_prefetch_desc(&tmq);
+    tma_prefetch_desc(&tmk);
+    tma_prefetch_desc(&tmv);
+    mbar_init(&bar.q_full, 1);
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(&bar.k_full[s], 1);
+      mbar_init(&bar.k_empty[s], 1);
+      mbar_init(&bar.v_full[s], 1);
+      mbar_init(&bar.v_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar.s_full[i], 1);
+      mbar_init(&bar.p_full[i], 128);
+    }
+    mbar_init(&bar.pv_done, 1);
+    mbar_init(&bar.o_full, 1);
+    mbar_init(&bar.drain, 1);
+    bar.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&bar.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+  volatile int* abort_flag = &bar.abort;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int last_q = 0;
+      int k_uses[Cfg::kStages], v_uses[Cfg::kStages];
+      for (int s = 0; s < Cfg::kStages; ++s) k_uses[s] = v_uses[s] = 0;
+      bool ok = true;
+      mbar_arrive_expect_tx(&bar.q_full, Cfg::kQBytes);
+      for (int c = 0; c < Cfg::kChunks; ++c)
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_3d(sQ + c * (kBM * 128) + hf * (64 * 128), &tmq, &bar.q_full, c * 64, t * kBM + hf * 64, bh);
+      last_q = 1;
+      for (int j = 0; j < n_iter && ok; ++j) {
+        const int kb = DENSE ? j : (tile_col[list_base + j] >> 2);
+        if (kb < 0 || kb >= nB) {
+          report(dev_status, FVA_DEVERR_BAD_LIST);
+          *abort_flag = 1;
+          break;
+        }
+        const int s = j % Cfg::kStages;
+        const uint32_t use = static_cast<uint32_t>(j / Cfg::kStages);
+        if (j >= Cfg::kStages && !mbar_wait(&bar.k_empty[s], (use - 1) & 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&bar.k_full[s], Cfg::kKVBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_3d(sK + s * Cfg::kKVBytes + c * (kBN * 128), &tmk, &bar.k_full[s], c * 64, kb * kBN, bh);
+        ++k_uses[s];
+        if (j >= Cfg::kStages && !mbar_wait(&bar.v_empty[s], (use - 1) & 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&bar.v_full[s], Cfg::kKVBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          tma_load_3d(sV + s * Cfg::kKVBytes + c * (kBN * 128), &tmv, &bar.v_full[s], c * 64, kb * kBN, bh);
+        ++v_uses[s];
+      }
+      if (!ok) {
+        report(dev_status, FVA_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      if (*abort_flag) {
+        // drain: wait (bounded) for the last load issued into every buffer
+        volatile int never = 0;
+        if (last_q) mbar_wait(&bar.q_full, 0, &never, 100000000ull);
+        for (int s = 0; s < Cfg::kStages; ++s) {
+          if (k_uses[s] > 0) mbar_wait(&bar.k_full[s], (k_uses[s] - 1) & 1, &never, 100000000ull);
+          if (v_uses[s] > 0) mbar_wait(&bar.v_full[s], (v_uses[s] - 1) & 1, &never, 100000000ull);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);
+      bool ok = mbar_wait(&bar.q_full, 0, abort_flag, kWaitLimitNs);
+      bool issued = false;
+      auto issue_pv = [&](int i) -> bool {
+        const int sb = i & 1;
+        const int s = i % Cfg::kStages;
+        if (!mbar_wait(&bar.p_full[sb], (i >> 1) & 1, abort_flag, kWaitLimitNs)) return false;
+        if (!mbar_wait(&bar.v_full[s], (i / Cfg::kStages) & 1, abort_flag, kWaitLimitNs)) return false;
+        tc_fence_after();
+        const uint32_t v_base = smem_u32(sV + s * Cfg::kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t bdesc = sdesc_sw128(v_base + kk * 2048, kBN * 128, 1024);
+          mma_ts(tmem + Cfg::kOCol, tmem + sb * 64 + kk * 8, bdesc, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&bar.v_empty[s]);
+        tc_commit(&bar.pv_done);
+        return true;
+      };
+      if (ok) tc_fence_after();
+      for (int j = 0; j < n_iter && ok; ++j) {
+        const int s = j % Cfg::kStages;
+        const int sb = j & 1;
+        if (!mbar_wait(&bar.k_full[s], (j / Cfg::kStages) & 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t q_base = smem_u32(sQ);
+        const uint32_t k_base = smem_u32(sK + s * Cfg::kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int c = kk >> 2;
+          const uint32_t ko = (kk & 3) * 32;
+          const uint64_t adesc = sdesc_sw128(q_base + c * (kBM * 128) + ko, 16, 1024);
+          const uint64_t bdesc = sdesc_sw128(k_base + c * (kBN * 128) + ko, 16, 1024);
+          mma_ss(tmem + sb * 64, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        issued = true;
+        tc_commit(&bar.k_empty[s]);
+        tc_commit(&bar.s_full[sb]);
+        if (j >= 1 && !issue_pv(j - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok && n_iter > 0) ok = issue_pv(n_iter - 1);
+      if (ok) {
+        tc_commit(&bar.o_full);
+      } else {
+        report(dev_status, FVA_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+        if (issued) {
+          // drain every MMA issued so far before TMEM is freed
+          volatile int never = 0;
+          tc_commit(&bar.drain);
+          mbar_wait(&bar.drain, 0, &never, 100000000ull);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warps 0-3
+    const int row = warp * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int half = warp >> 1;
+    float m_ref = -INFINITY;
+    float l_sum = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < n_iter; ++j) {
+      const int entry = DENSE ? ((j << 2) | 3) : tile_col[list_base + j];
+      const int kb = entry >> 2;
+      const bool keep = (entry >> half) & 1;
+      const int sb = j & 1;
+      if (!warp_wait(&bar.s_full[sb], (j >> 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t pk[32];
+      if (keep) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(lane_base + sb * 64, r0);
+        tmem_ld32(lane_base + sb * 64 + 32, r1);
+        const int nvalid = (kb == nB - 1) ? (N - kb * kBN) : kBN;
+        float x[64];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          x[c] = (c < nvalid) ? __uint_as_float(r0[c]) * scale_log2 : -INFINITY;
+          x[c + 32] = (c + 32 < nvalid) ? __uint_as_float(r1[c]) * scale_log2 : -INFINITY;
+        }
+        float mx = x[0];
+#pragma unroll
+        for (int c = 1; c < 64; ++c) mx = fmaxf(mx, x[c]);
+        const float m_new = fmaxf(m_ref, mx);
+        const bool need = m_new > m_ref + 8.0f;
+        const bool need_o = need && (l_sum > 0.0f);
+        if (__any_sync(0xffffffffu, need_o)) {
+          // O holds rows rescaled to the old maximum: wait for the PV of step j-1, then
+          // O_row *= 2^(m_ref - m_new) for the rows whose maximum moved.
+          if (!warp_wait(&bar.pv_done, (j - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float alpha = need_o ? ex2_approx(m_ref - m_new) : 1.0f;
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + Cfg::kOCol + cc * 32, o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(lane_base + Cfg::kOCol + cc * 32, o);
+          }
+        }
+        if (need) {
+          l_sum *= ex2_approx(m_ref - m_new);
+          m_ref = m_new;
+        }
+        float ls = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float p0 = ex2_approx(x[2 * c] - m_ref);
+          const float p1 = ex2_approx(x[2 * c + 1] - m_ref);
+          ls += p0 + p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        l_sum += ls;
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+      }
+      tmem_st32(lane_base + sb * 64, pk);
+      tc_fence_before();
+      mbar_arrive(&bar.p_full[sb]);
+    }
+    // ------------------------------------------------------------------ epilogue
+    if (ok && !warp_wait(&bar.o_full, 0, abort_flag)) ok = false;
+    if (!ok) {
+      report(dev_status, FVA_DEVERR_TIMEOUT);
+      *abort_flag = 1;
+    } else {
+      tc_fence_after();
+      const float inv_l = l_sum > 0.0f ? 1.0f / l_sum : 0.0f;
+      const int grow = t * kBM + row;
+      const bool valid = grow < N && n_iter > 0;
+      uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<int64_t>(bh) * N + grow) * D);
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(lane_base + Cfg::kOCol + cc * 32, o);
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
+        if (valid) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[cc * 4 + q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        }
+      }
+      if (n_iter == 0 && grow < N) {
+        for (int q = 0; q < D / 8; ++q) dst[q] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D map over a [B*H, N, d] bf16 tensor, box = 64 elements (128 B) x 64 rows x 1.
+static bool make_map(CUtensorMap* map, const void* base, int64_t BH, int64_t N, int64_t d) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(N * d * 2)};
+  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, bool DENSE>
+static cudaError_t launch_attn_t(const Dims& Dm, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                 const fva_mask* m, void* o, float scale_log2, int32_t* dev_status, cudaStream_t st) {
+  const size_t smem = attn_smem_bytes<D>();
+  cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<D, DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(Dm.tiles);
+  attn_bf16_kernel<D, DENSE><<<grid, kAttnThreads, smem, st>>>(
+      mq, mk, mv, static_cast<__nv_bfloat16*>(o), DENSE ? nullptr : m->tile_ptr, DENSE ? nullptr : m->tile_col,
+      DENSE ? nullptr : m->worklist, static_cast<int>(Dm.N), static_cast<int>(Dm.nB), static_cast<int>(Dm.nPairs),
+      scale_log2, dev_status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_bf16(const Dims& Dm, const void* q, const void* k, const void* v, const fva_mask* m,
+                             bool dense, void* o, float scale, int32_t* dev_status, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, Dm.BH, Dm.N, Dm.d) || !make_map(&mk, k, Dm.BH, Dm.N, Dm.d) ||
+      !make_map(&mv, v, Dm.BH, Dm.N, Dm.d))
+    return cudaErrorInvalidValue;
+  const float scale_log2 = scale * 1.4426950408889634f;
+  if (Dm.d == 128) {
+    return dense ? launch_attn_t<128, true>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st)
+                 : launch_attn_t<128, false>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st);
+  }
+  return dense ? launch_attn_t<64, true>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st)
+               : launch_attn_t<64, false>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st);
+}
+
+}  // namespace fva

@@ -1,0 +1,247 @@
+// Hilbert token order, token reorder with fused float64 block mean-pooling, and its
+// inverse ("video-aware block organization", aixai.ru FVAttn blog, "Sparse-routing
+// frontend"; pooled Q/K, PaperDaily FVAttn article, 方法揭秘).
+//
+// The permute kernels are pure data movement and HBM-bound: each CTA owns one
+// 64-token block of one (b, h), so every 16-byte vector is read once and written once,
+// and the block's pooled row is reduced inside the CTA (no atomics).
+#include "fva_internal.cuh"
+
+namespace fva {
+
+// ---------------------------------------------------------------------------------
+// Hilbert order of one frame
+// ---------------------------------------------------------------------------------
+
+// Cell (x, y) at distance t along the Hilbert curve of side 2^m. Walks the base-4
+// digits of t from the least significant: each digit picks a quadrant of the current
+// sub-square, and the cells found so far are reflected into that quadrant's
+// orientation (lower-left: swap axes; lower-right: reflect about the anti-diagonal).
+__device__ __forceinline__ void hilbert_cell(int m, uint32_t t, int* px, int* py) {
+  int x = 0, y = 0;
+  for (int level = 0; level < m; ++level) {
+    const int side = 1 << level;
+    const int hi = (t >> 1) & 1;           // right half?
+    const int up = (t ^ hi) & 1;           // upper half?
+    if (!up) {
+      if (hi) {
+        x = side - 1 - x;
+        y = side - 1 - y;
+      }
+      const int tmp = x;
+      x = y;
+      y = tmp;
+    }
+    x += side * hi;
+    y += side * up;
+    t >>= 2;
+  }
+  *px = x;
+  *py = y;
+}
+
+// One CTA: enumerate the curve of the enclosing square in order, keep in-grid cells
+// (block-wide scan for their output slots) and write frame 0's order to perm[0, HW).
+__global__ void __launch_bounds__(1024) hilbert_frame_kernel(int m, int Hg, int Wg, int32_t* perm) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  const uint32_t total = 1u << (2 * m);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (uint32_t base = 0; base < total; base += blockDim.x) {
+    const uint32_t t = base + threadIdx.x;
+    int x = 0, y = 0, valid = 0;
+    if (t < total) {
+      hilbert_cell(m, t, &x, &y);
+      valid = (x < Wg && y < Hg) ? 1 : 0;
+    }
+    const uint32_t ballot = __ballot_sync(0xffffffffu, valid);
+    const int in_warp = __popc(ballot & ((1u << lane) - 1u));
+    if (lane == 0) warp_tot[warp] = __popc(ballot);
+    __syncthreads();
+    int before = 0, all = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
+      const int c = warp_tot[w];
+      if (w < warp) before += c;
+      all += c;
+    }
+    const int pos = carry + before + in_warp;
+    if (valid) perm[pos] = y * Wg + x;
+    __syncthreads();
+    if (threadIdx.x == 0) carry += all;
+    __syncthreads();
+  }
+}
+
+// Replicate frame 0's order over the T frames and build the inverse.
+__global__ void hilbert_frames_kernel(int64_t HW, int64_t N, int32_t* perm, int32_t* inv) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < N;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / HW;
+    const int32_t cell = perm[i - t * HW];
+    const int64_t src = t * HW + cell;
+    if (t > 0) perm[i] = static_cast<int32_t>(src);
+    inv[src] = static_cast<int32_t>(i);
+  }
+}
+
+cudaError_t launch_hilbert_perm(const Dims& D, int T, int Hg, int Wg, int32_t* perm, int32_t* inv,
+                                cudaStream_t st) {
+  int m = 0;
+  while ((1 << m) < (Hg > Wg ? Hg : Wg)) ++m;
+  hilbert_frame_kernel<<<1, 1024, 0, st>>>(m, Hg, Wg, perm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t HW = static_cast<int64_t>(Hg) * Wg;
+  int grid = static_cast<int>((D.N + 255) / 256);
+  if (grid > 148 * 16) grid = 148 * 16;
+  // frame 0 entries are read by every frame; the kernel only rewrites frames t > 0, so
+  // the reads of perm[0, HW) never race with writes.
+  hilbert_frames_kernel<<<grid, 256, 0, st>>>(HW, D.N, perm, inv);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------------
+// Reorder / pool
+// ---------------------------------------------------------------------------------
+
+template <typename T>
+__device__ __forceinline__ void add_vec(double* acc, const uint4& v);
+
+template <>
+__device__ __forceinline__ void add_vec<__nv_bfloat16>(double* acc, const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] += static_cast<double>(__uint_as_float(w[i] << 16));
+    acc[2 * i + 1] += static_cast<double>(__uint_as_float(w[i] & 0xFFFF0000u));
+  }
+}
+template <>
+__device__ __forceinline__ void add_vec<float>(double* acc, const uint4& v) {
+  acc[0] += static_cast<double>(__uint_as_float(v.x));
+  acc[1] += static_cast<double>(__uint_as_float(v.y));
+  acc[2] += static_cast<double>(__uint_as_float(v.z));
+  acc[3] += static_cast<double>(__uint_as_float(v.w));
+}
+
+constexpr int kReorderThreads = 256;
+
+// MODE 0: forward permute [B,N,H,d] -> [B,H,N,d] (+ pool)
+// MODE 1: inverse permute [B,H,N,d] -> [B,N,H,d]
+// MODE 2: pool only, input already [B,H,N,d]
+// One CTA per (block a, head h, batch b). VPR = 16-byte vectors per (token, head) row.
+template <typename T, int MODE, bool POOL>
+__global__ void __launch_bounds__(kReorderThreads) reorder_kernel(
+    const uint8_t* __restrict__ x_in, uint8_t* __restrict__ x_out, double* __restrict__ pooled,
+    const int32_t* __restrict__ perm, int N, int H, int vpr) {
+  constexpr int EPV = 16 / sizeof(T);  // elements per 16-byte vector
+  extern __shared__ double red[];      // [rows_per_pass][vpr * EPV] when POOL
+  const int a = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int64_t row_bytes = static_cast<int64_t>(vpr) * 16;
+  const int v = threadIdx.x % vpr;
+  const int r0 = threadIdx.x / vpr;
+  const int rpp = kReorderThreads / vpr;  // rows per pass
+  const bool active = r0 < rpp;           // threads beyond rpp*vpr idle
+  const int row_lo = a * kBlock;
+  const int n_valid = min(kBlock, N - row_lo);
+  double acc[EPV];
+#pragma unroll
+  for (int i = 0; i < EPV; ++i) acc[i] = 0.0;
+
+  if (active) {
+    constexpr int kMaxPass = 16;  // rpp >= 4 (vpr <= 64), so 64/rpp <= 16
+    uint4 buf[kMaxPass];
+    const int n_pass = (kBlock + rpp - 1) / rpp;
+#pragma unroll
+    for (int ps = 0; ps < kMaxPass; ++ps) {
+      if (ps < n_pass) {
+        const int r = r0 + ps * rpp;
+        if (r < n_valid) {
+          const int i = row_lo + r;
+          const uint8_t* src;
+          if (MODE == 0) {
+            src = x_in + ((static_cast<int64_t>(b) * N + perm[i]) * H + h) * row_bytes;
+          } else {
+            src = x_in + ((static_cast<int64_t>(b) * H + h) * N + i) * row_bytes;
+          }
+          buf[ps] = __ldg(reinterpret_cast<const uint4*>(src) + v);
+        }
+      }
+    }
+#pragma unroll
+    for (int ps = 0; ps < kMaxPass; ++ps) {
+      if (ps < n_pass) {
+        const int r = r0 + ps * rpp;
+        if (r < n_valid) {
+          const int i = row_lo + r;
+          if (MODE != 2) {
+            uint8_t* dst;
+            if (MODE == 0) {
+              dst = x_out + ((static_cast<int64_t>(b) * H + h) * N + i) * row_bytes;
+            } else {
+              dst = x_out + ((static_cast<int64_t>(b) * N + perm[i]) * H + h) * row_bytes;
+            }
+            reinterpret_cast<uint4*>(dst)[v] = buf[ps];
+          }
+          if (POOL) add_vec<T>(acc, buf[ps]);
+        }
+      }
+    }
+  }
+  if (POOL) {
+    const int width = vpr * EPV;  // = d
+    if (active) {
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) red[r0 * width + v * EPV + e] = acc[e];
+    }
+    __syncthreads();
+    // column sums over the rpp partial rows, fixed order
+    for (int c = threadIdx.x; c < width; c += kReorderThreads) {
+      double s = 0.0;
+      for (int r = 0; r < rpp; ++r) s += red[r * width + c];
+      pooled[((static_cast<int64_t>(b) * H + h) * gridDim.x + a) * width + c] = s / static_cast<double>(n_valid);
+    }
+  }
+}
+
+template <typename T>
+static cudaError_t launch_reorder_t(const Dims& D, const void* x_in, void* x_out, double* pooled,
+                                    const int32_t* perm, int mode, cudaStream_t st) {
+  const int vpr = static_cast<int>(D.d * sizeof(T) / 16);
+  const int rpp = kReorderThreads / vpr;
+  const dim3 grid(static_cast<unsigned>(D.nB), static_cast<unsigned>(D.H), static_cast<unsigned>(D.B));
+  const size_t smem = pooled ? static_cast<size_t>(rpp) * D.d * sizeof(double) : 0;
+  const uint8_t* in = static_cast<const uint8_t*>(x_in);
+  uint8_t* out = static_cast<uint8_t*>(x_out);
+  const int N = static_cast<int>(D.N), H = static_cast<int>(D.H);
+  if (mode == 0 && pooled) {
+    cudaFuncSetAttribute(reorder_kernel<T, 0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
+    reorder_kernel<T, 0, true><<<grid, kReorderThreads, smem, st>>>(in, out, pooled, perm, N, H, vpr);
+  } else if (mode == 0) {
+    reorder_kernel<T, 0, false><<<grid, kReorderThreads, 0, st>>>(in, out, nullptr, perm, N, H, vpr);
+  } else if (mode == 1) {
+    reorder_kernel<T, 1, false><<<grid, kReorderThreads, 0, st>>>(in, out, nullptr, perm, N, H, vpr);
+  } else {
+    cudaFuncSetAttribute(reorder_kernel<T, 2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
+    reorder_kernel<T, 2, true><<<grid, kReorderThreads, smem, st>>>(in, nullptr, pooled, nullptr, N, H, vpr);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reorder(const Dims& D, const void* x_in, void* x_out, double* pooled,
+                           const int32_t* perm, int direction, cudaStream_t st) {
+  const int mode = direction == FVA_FWD ? 0 : 1;
+  if (D.esize == 2) return launch_reorder_t<__nv_bfloat16>(D, x_in, x_out, pooled, perm, mode, st);
+  return launch_reorder_t<float>(D, x_in, x_out, pooled, perm, mode, st);
+}
+
+cudaError_t launch_pool(const Dims& D, const void* x_bhnd, double* pooled, cudaStream_t st) {
+  if (D.esize == 2) return launch_reorder_t<__nv_bfloat16>(D, x_bhnd, nullptr, pooled, nullptr, 2, st);
+  return launch_reorder_t<float>(D, x_bhnd, nullptr, pooled, nullptr, 2, st);
+}
+
+}  // namespace fva

@@ -1,0 +1,692 @@
+// Top-p block routing with a Top-k safety floor, CSR mask, per-head kept counts,
+// tile lists and the longest-first work list.
+//
+// Method (aixai.ru FVAttn blog, "Top-p vs Top-k" and "Sparse-routing frontend";
+// PaperDaily FVAttn article, 方法揭秘 and 龙迷三问): block importance from pooled Q/K,
+// keep key blocks in importance order until the cumulative importance reaches p, and
+// never fewer than k_floor blocks.
+//
+// Kernels (all float64 where a value decides the mask):
+//   route_scores_kernel   S = pooled_q pooled_k^T / sqrt(d), register-tiled DFMA GEMM
+//   route_select_kernel   one warp per row: softmax, bucket refinement to the cut,
+//                         exact (logit desc, index asc) order inside the last bucket,
+//                         kept bitmask, kept count, per-tile union cost
+//   finish_kernel         row_ptr / tile_ptr scans, head_kept, per-head load
+//   order_*_kernel        work list (natural, global LPT, head-grouped LPT)
+//   emit_kernel           col_idx (ascending) and tile_col (union + membership bits)
+#include <math.h>
+
+#include "fva_internal.cuh"
+
+namespace fva {
+
+// ---------------------------------------------------------------------------------
+// Block logits
+// ---------------------------------------------------------------------------------
+constexpr int kST = 64;  // output tile (rows and columns)
+constexpr int kSK = 16;  // d-chunk staged per step
+
+__global__ void __launch_bounds__(256) route_scores_kernel(const double* __restrict__ pq,
+                                                           const double* __restrict__ pk,
+                                                           double* __restrict__ S, int nB, int d,
+                                                           double sqrt_d) {
+  __shared__ __align__(16) double As[kSK][kST];
+  __shared__ __align__(16) double Bs[kSK][kST];
+  const int bh = blockIdx.z;
+  const int a0 = blockIdx.y * kST, b0 = blockIdx.x * kST;
+  const double* Q = pq + static_cast<int64_t>(bh) * nB * d;
+  const double* K = pk + static_cast<int64_t>(bh) * nB * d;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  double acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+
+  for (int i0 = 0; i0 < d; i0 += kSK) {
+    for (int e = threadIdx.x; e < kST * kSK; e += 256) {
+      const int r = e / kSK, c = e % kSK;
+      const int ga = a0 + r, gb = b0 + r;
+      As[c][r] = (ga < nB && i0 + c < d) ? Q[static_cast<int64_t>(ga) * d + i0 + c] : 0.0;
+      Bs[c][r] = (gb < nB && i0 + c < d) ? K[static_cast<int64_t>(gb) * d + i0 + c] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int c = 0; c < kSK; ++c) {
+      const double2 a01 = *reinterpret_cast<const double2*>(&As[c][ty * 4]);
+      const double2 a23 = *reinterpret_cast<const double2*>(&As[c][ty * 4 + 2]);
+      const double2 b01 = *reinterpret_cast<const double2*>(&Bs[c][tx * 4]);
+      const double2 b23 = *reinterpret_cast<const double2*>(&Bs[c][tx * 4 + 2]);
+      const double av[4] = {a01.x, a01.y, a23.x, a23.y};
+      const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fma(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int a = a0 + ty * 4 + i;
+    if (a >= nB) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int b = b0 + tx * 4 + j;
+      if (b < nB) S[(static_cast<int64_t>(bh) * nB + a) * nB + b] = acc[i][j] / sqrt_d;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// Selection
+// ---------------------------------------------------------------------------------
+constexpr int kNBK = 128;                       // buckets per refinement level
+constexpr int kMaxLevels = 12;
+constexpr double kFix = 4503599627370496.0;     // 2^52: fixed-point unit of importance
+
+struct WarpArena {
+  double* e;          // [nB] exp(s - max)
+  uint64_t* hw;       // [kNBK] bucket mass (fixed point)
+  int32_t* list;      // [nB] candidate block indices
+  int32_t* hcnt;      // [kNBK] bucket counts
+  uint32_t* words;    // [nWords] kept bitmask of the row
+};
+
+__host__ __device__ inline size_t warp_arena_bytes(int nB, int nWords) {
+  size_t b = 0;
+  b += align_up(static_cast<size_t>(nB) * 8, 16);
+  b += kNBK * 8;
+  b += align_up(static_cast<size_t>(nB) * 4, 16);
+  b += kNBK * 4;
+  b += align_up(static_cast<size_t>(nWords) * 4, 16);
+  return b;
+}
+
+__device__ inline WarpArena make_arena(uint8_t* base, int nB, int nWords) {
+  WarpArena A;
+  size_t off = 0;
+  A.e = reinterpret_cast<double*>(base + off);
+  off += align_up(static_cast<size_t>(nB) * 8, 16);
+  A.hw = reinterpret_cast<uint64_t*>(base + off);
+  off += kNBK * 8;
+  A.list = reinterpret_cast<int32_t*>(base + off);
+  off += align_up(static_cast<size_t>(nB) * 4, 16);
+  A.hcnt = reinterpret_cast<int32_t*>(base + off);
+  off += kNBK * 4;
+  A.words = reinterpret_cast<uint32_t*>(base + off);
+  return A;
+}
+
+// (s_j, j) precedes (s_i, i) in the routing order: larger logit, or equal logit and
+// lower block index.
+__device__ __forceinline__ bool precedes(double sj, int j, double si, int i) {
+  return sj > si || (sj == si && j < i);
+}
+
+__device__ __forceinline__ uint64_t fixed_mass(double e, double Z) {
+  return static_cast<uint64_t>((e / Z) * kFix);
+}
+
+struct Pivot {
+  int found;   // 0: the mass target is never reached (keep everything)
+  int L;       // 1-based position of the pivot in the routing order
+  double s;    // pivot logit
+  int b;       // pivot block
+};
+
+// Find the pivot of the routing order for one row.
+// by_mass: the first position whose cumulative fixed-point mass reaches `pth`
+// (= p * 2^52); otherwise the position `cnt_target` (1-based) by count.
+__device__ Pivot select_pivot(const double* __restrict__ srow, const WarpArena& A, int nB, double smax,
+                              double smin, double Z, bool by_mass, double pth, int cnt_target) {
+  const int lane = threadIdx.x & 31;
+  uint64_t above_w = 0;
+  int above_c = 0;
+  double lo = smin, hi = smax;
+  int c = nB;            // candidates
+  bool implicit = true;  // candidates are all blocks [0, nB)
+  for (int level = 0; level < kMaxLevels; ++level) {
+    if (c <= 32 || !(hi > lo)) break;
+    const double kappa = static_cast<double>(kNBK) / (hi - lo);
+    for (int i = lane; i < kNBK; i += 32) {
+      A.hcnt[i] = 0;
+      A.hw[i] = 0;
+    }
+    __syncwarp();
+    for (int i = lane; i < c; i += 32) {
+      const int b = implicit ? i : A.list[i];
+      const double s = srow[b];
+      int bk = static_cast<int>((hi - s) * kappa);
+      bk = bk < 0 ? 0 : (bk >= kNBK ? kNBK - 1 : bk);
+      atomicAdd(&A.hcnt[bk], 1);
+      if (by_mass) atomicAdd(reinterpret_cast<unsigned long long*>(&A.hw[bk]),
+                             static_cast<unsigned long long>(fixed_mass(A.e[b], Z)));
+    }
+    __syncwarp();
+    // lane owns buckets 4*lane .. 4*lane+3
+    int cnt4[4];
+    uint64_t w4[4];
+    int csum = 0;
+    uint64_t wsum = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      cnt4[q] = A.hcnt[4 * lane + q];
+      w4[q] = A.hw[4 * lane + q];
+      csum += cnt4[q];
+      wsum += w4[q];
+    }
+    // exclusive prefix over lanes
+    int cpre = csum;
+    uint64_t wpre = wsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int cn = __shfl_up_sync(0xffffffffu, cpre, o);
+      const uint64_t wn = __shfl_up_sync(0xffffffffu, wpre, o);
+      if (lane >= o) {
+        cpre += cn;
+        wpre += wn;
+      }
+    }
+    cpre -= csum;
+    wpre -= wsum;
+    // first bucket (lowest index = highest logits) where the running total reaches the target
+    int hit = kNBK;
+    int hit_c_before = 0;
+    uint64_t hit_w_before = 0;
+    {
+      int cc = cpre;
+      uint64_t ww = wpre;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const bool reach = by_mass ? (static_cast<double>(above_w + ww + w4[q]) >= pth)
+                                   : (above_c + cc + cnt4[q] >= cnt_target);
+        if (reach && hit == kNBK) {
+          hit = 4 * lane + q;
+          hit_c_before = cc;
+          hit_w_before = ww;
+        }
+        cc += cnt4[q];
+        ww += w4[q];
+      }
+    }
+    // lowest lane with a hit decides
+    const unsigned hmask = __ballot_sync(0xffffffffu, hit < kNBK);
+    if (hmask == 0) {
+      Pivot none;
+      none.found = 0;
+      none.L = nB;
+      none.s = smin;
+      none.b = nB - 1;
+      return none;  // mass target not reached by the whole row
+    }
+    const int src = __ffs(hmask) - 1;
+    const int B = __shfl_sync(0xffffffffu, hit, src);
+    above_c += __shfl_sync(0xffffffffu, hit_c_before, src);
+    above_w += __shfl_sync(0xffffffffu, hit_w_before, src);
+    // compact the candidates of bucket B (ascending block index is kept)
+    int newc = 0;
+    double nlo = INFINITY, nhi = -INFINITY;
+    for (int i0 = 0; i0 < c; i0 += 32) {
+      const int i = i0 + lane;
+      int b = -1;
+      bool in = false;
+      double s = 0.0;
+      if (i < c) {
+        b = implicit ? i : A.list[i];
+        s = srow[b];
+        int bk = static_cast<int>((hi - s) * kappa);
+        bk = bk < 0 ? 0 : (bk >= kNBK ? kNBK - 1 : bk);
+        in = (bk == B);
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, in);
+      __syncwarp();
+      if (in) {
+        A.list[newc + __popc(m & ((1u << lane) - 1u))] = b;
+        nlo = fmin(nlo, s);
+        nhi = fmax(nhi, s);
+      }
+      newc += __popc(m);
+      __syncwarp();
+    }
+    c = newc;
+    implicit = false;
+    lo = warp_min_d(nlo);
+    hi = warp_max_d(nhi);
+  }
+  if (implicit) {
+    for (int i = lane; i < c; i += 32) A.list[i] = i;
+    __syncwarp();
+  }
+  // exact order inside the remaining candidates: rank and inclusive cumulative mass
+  int best_rank = 0x7fffffff;
+  int best_b = -1;
+  double best_s = 0.0;
+  for (int i0 = 0; i0 < c; i0 += 32) {
+    const int i = i0 + lane;
+    if (i < c) {
+      const int bi = A.list[i];
+      const double si = srow[bi];
+      int rank = 0;
+      uint64_t cw = 0;
+      for (int j = 0; j < c; ++j) {
+        const int bj = A.list[j];
+        const double sj = srow[bj];
+        if (precedes(sj, bj, si, bi)) {
+          ++rank;
+          if (by_mass) cw += fixed_mass(A.e[bj], Z);
+        }
+      }
+      bool ok;
+      if (by_mass) {
+        cw += fixed_mass(A.e[bi], Z);
+        ok = static_cast<double>(above_w + cw) >= pth;
+      } else {
+        ok = (above_c + rank + 1 == cnt_target);
+      }
+      if (ok && rank < best_rank) {
+        best_rank = rank;
+        best_b = bi;
+        best_s = si;
+      }
+    }
+  }
+  // warp argmin over rank
+  int r = best_rank;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) r = min(r, __shfl_xor_sync(0xffffffffu, r, o));
+  const unsigned who = __ballot_sync(0xffffffffu, best_rank == r && best_b >= 0);
+  Pivot pv;
+  if (who == 0) {
+    pv.found = 0;  // mass target not reached (truncated total below p)
+    pv.L = nB;
+    pv.s = smin;
+    pv.b = nB - 1;
+    return pv;
+  }
+  const int src = __ffs(who) - 1;
+  pv.found = 1;
+  pv.L = above_c + r + 1;
+  pv.b = __shfl_sync(0xffffffffu, best_b, src);
+  pv.s = __shfl_sync(0xffffffffu, best_s, src);
+  return pv;
+}
+
+// grid: (ceil(nB / rows_per_cta), BH); block: 32 * rows_per_cta (rows_per_cta even)
+__global__ void route_select_kernel(const double* __restrict__ S, int nB, int nWords, int nPairs,
+                                    double p, int k_floor, uint32_t* __restrict__ bits,
+                                    int32_t* __restrict__ row_cnt, int32_t* __restrict__ tile_cost,
+                                    int32_t* dev_status) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rows_per_cta = blockDim.x >> 5;
+  const int bh = blockIdx.y;
+  const int a0 = blockIdx.x * rows_per_cta;
+  const int a = a0 + warp;
+  const size_t arena = warp_arena_bytes(nB, nWords);
+  WarpArena A = make_arena(smem_raw + arena * warp, nB, nWords);
+
+  if (a < nB) {
+    const int64_t row = static_cast<int64_t>(bh) * nB + a;
+    const double* srow = S + row * nB;
+    double smax = -INFINITY, smin = INFINITY;
+    for (int b = lane; b < nB; b += 32) {
+      const double s = srow[b];
+      smax = fmax(smax, s);
+      smin = fmin(smin, s);
+    }
+    smax = warp_max_d(smax);
+    smin = warp_min_d(smin);
+    double z = 0.0;
+    for (int b = lane; b < nB; b += 32) {
+      const double e = exp(srow[b] - smax);
+      A.e[b] = e;
+      z += e;
+    }
+    const double Z = warp_sum_d(z);
+    __syncwarp();
+
+    const int L_k = k_floor < nB ? k_floor : nB;
+    bool all = (p >= 1.0) || (L_k >= nB);
+    Pivot pv;
+    pv.found = 0;
+    pv.L = nB;
+    pv.s = smin;
+    pv.b = nB - 1;
+    if (!all) {
+      pv = select_pivot(srow, A, nB, smax, smin, Z, true, p * kFix, 0);
+      if (!pv.found) {
+        all = true;
+      } else if (pv.L < L_k) {
+        pv = select_pivot(srow, A, nB, smax, smin, Z, false, 0.0, L_k);
+        if (!pv.found) all = true;
+      }
+    }
+    int kept = 0;
+    for (int k = 0; k < nWords; ++k) {
+      const int b = 32 * k + lane;
+      bool keep = false;
+      if (b < nB) keep = all || precedes(srow[b], b, pv.s, pv.b) || b == pv.b;
+      const unsigned w = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0) A.words[k] = w;
+      kept += __popc(w);
+    }
+    __syncwarp();
+    for (int k = lane; k < nWords; k += 32) bits[row * nWords + k] = A.words[k];
+    if (lane == 0) {
+      row_cnt[row] = kept;
+      if (kept != (all ? nB : pv.L)) report(dev_status, FVA_DEVERR_MASK);
+    }
+  }
+  __syncthreads();
+  // per-tile union cost for the pairs (2t, 2t+1) inside this CTA (a0 is even)
+  if ((warp & 1) == 0 && a < nB) {
+    const int t = a >> 1;
+    const bool has_b = (a + 1 < nB);
+    const WarpArena Bn = make_arena(smem_raw + arena * (warp + 1), nB, nWords);
+    int u = 0;
+    for (int k = lane; k < nWords; k += 32) u += __popc(A.words[k] | (has_b ? Bn.words[k] : 0u));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+    if (lane == 0) tile_cost[static_cast<int64_t>(bh) * nPairs + t] = u;
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// Scans, per-head counts
+// ---------------------------------------------------------------------------------
+// Exclusive scan of n int32 into out[0..n] by one 1024-thread block; returns total.
+__device__ int64_t block_exclusive_scan(const int32_t* __restrict__ in, int32_t* __restrict__ out,
+                                        int64_t n, int64_t* smem_warp /*[32]*/) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t chunk = (n + blockDim.x - 1) / blockDim.x;
+  const int64_t lo = tid * chunk;
+  const int64_t hi = lo + chunk < n ? lo + chunk : n;
+  int64_t local = 0;
+  for (int64_t i = lo; i < hi; ++i) local += in[i];
+  int64_t inc = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t v = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += v;
+  }
+  if (lane == 31) smem_warp[warp] = inc;
+  __syncthreads();
+  int64_t warp_base = 0, total = 0;
+  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
+    if (w < warp) warp_base += smem_warp[w];
+    total += smem_warp[w];
+  }
+  int64_t run = warp_base + inc - local;
+  for (int64_t i = lo; i < hi; ++i) {
+    out[i] = static_cast<int32_t>(run);
+    run += in[i];
+  }
+  if (tid == 0) out[n] = static_cast<int32_t>(total);
+  __syncthreads();
+  return total;
+}
+
+__global__ void __launch_bounds__(1024) finish_kernel(const int32_t* __restrict__ row_cnt, int64_t rows,
+                                                      const int32_t* __restrict__ tile_cost, int64_t tiles,
+                                                      int nB, int nPairs, int BH, int32_t* row_ptr,
+                                                      int32_t* tile_ptr, int64_t* head_kept, int64_t* head_load,
+                                                      int64_t capacity, int64_t tile_capacity,
+                                                      int32_t* dev_status) {
+  __shared__ int64_t sw[32];
+  int64_t total_rows = -1;
+  if (row_cnt) total_rows = block_exclusive_scan(row_cnt, row_ptr, rows, sw);
+  const int64_t total_tiles = block_exclusive_scan(tile_cost, tile_ptr, tiles, sw);
+  __syncthreads();
+  for (int bh = threadIdx.x; bh < BH; bh += blockDim.x) {
+    head_kept[bh] = static_cast<int64_t>(row_ptr[static_cast<int64_t>(bh + 1) * nB]) -
+                    row_ptr[static_cast<int64_t>(bh) * nB];
+    head_load[bh] = static_cast<int64_t>(tile_ptr[static_cast<int64_t>(bh + 1) * nPairs]) -
+                    tile_ptr[static_cast<int64_t>(bh) * nPairs];
+  }
+  if (threadIdx.x == 0) {
+    if (total_rows > capacity || total_tiles > tile_capacity) report(dev_status, FVA_DEVERR_MASK);
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// Work list orders
+// ---------------------------------------------------------------------------------
+__global__ void order_natural_kernel(int32_t* worklist, int64_t tiles) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < tiles;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    worklist[i] = static_cast<int32_t>(i);
+}
+
+// rank(t) = #{t' : cost' > cost or (cost' == cost and t' < t)}; worklist[rank] = t
+__global__ void __launch_bounds__(256) order_lpt_kernel(const int32_t* __restrict__ cost, int64_t tiles,
+                                                        int32_t* worklist) {
+  __shared__ int32_t sc[2048];
+  const int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int32_t ct = t < tiles ? cost[t] : 0;
+  int64_t rank = 0;
+  for (int64_t base = 0; base < tiles; base += 2048) {
+    const int64_t n = tiles - base < 2048 ? tiles - base : 2048;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) sc[i] = cost[base + i];
+    __syncthreads();
+    if (t < tiles) {
+      for (int i = 0; i < n; ++i) {
+        const int32_t c = sc[i];
+        rank += (c > ct) || (c == ct && base + i < t);
+      }
+    }
+  }
+  if (t < tiles) worklist[rank] = static_cast<int32_t>(t);
+}
+
+// One CTA per (b, h): heads ordered by load desc (index asc), tiles of a head by cost desc
+// (index asc).
+__global__ void __launch_bounds__(256) order_head_lpt_kernel(const int32_t* __restrict__ cost,
+                                                             const int64_t* __restrict__ head_load, int BH,
+                                                             int nPairs, int32_t* worklist) {
+  extern __shared__ int32_t sc[];  // [nPairs]
+  __shared__ int64_t head_rank;
+  const int bh = blockIdx.x;
+  if (threadIdx.x == 0) {
+    const int64_t my = head_load[bh];
+    int64_t r = 0;
+    for (int j = 0; j < BH; ++j) {
+      const int64_t l = head_load[j];
+      r += (l > my) || (l == my && j < bh);
+    }
+    head_rank = r;
+  }
+  for (int i = threadIdx.x; i < nPairs; i += blockDim.x) sc[i] = cost[static_cast<int64_t>(bh) * nPairs + i];
+  __syncthreads();
+  for (int t = threadIdx.x; t < nPairs; t += blockDim.x) {
+    const int32_t ct = sc[t];
+    int r = 0;
+    for (int i = 0; i < nPairs; ++i) {
+      const int32_t c = sc[i];
+      r += (c > ct) || (c == ct && i < t);
+    }
+    worklist[head_rank * nPairs + r] = bh * nPairs + t;
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// Emission of col_idx and tile_col from the bitmasks
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ int warp_exclusive_scan_i(int v, int* total) {
+  const int lane = threadIdx.x & 31;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  *total = __shfl_sync(0xffffffffu, inc, 31);
+  return inc - v;
+}
+
+__global__ void __launch_bounds__(256) emit_kernel(const uint32_t* __restrict__ bits, int nB, int nWords,
+                                                   int nPairs, int64_t tiles, const int32_t* __restrict__ row_ptr,
+                                                   const int32_t* __restrict__ tile_ptr, int32_t* col_idx,
+                                                   int32_t* tile_col, int write_rows) {
+  const int lane = threadIdx.x & 31;
+  const int64_t tile = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (tile >= tiles) return;
+  const int64_t bh = tile / nPairs;
+  const int t = static_cast<int>(tile - bh * nPairs);
+  const int64_t rA = bh * nB + 2 * t;
+  const bool hasB = 2 * t + 1 < nB;
+  const int64_t rB = rA + 1;
+  const int64_t baseA = row_ptr[rA];
+  const int64_t baseB = hasB ? row_ptr[rB] : 0;
+  const int64_t baseT = tile_ptr[tile];
+  int runA = 0, runB = 0, runT = 0;
+  for (int k0 = 0; k0 < nWords; k0 += 32) {
+    const int k = k0 + lane;
+    const uint32_t wa = k < nWords ? bits[rA * nWords + k] : 0u;
+    const uint32_t wb = (hasB && k < nWords) ? bits[rB * nWords + k] : 0u;
+    const uint32_t wu = wa | wb;
+    int totA, totB, totU;
+    const int oa = warp_exclusive_scan_i(__popc(wa), &totA);
+    const int ob = warp_exclusive_scan_i(__popc(wb), &totB);
+    const int ou = warp_exclusive_scan_i(__popc(wu), &totU);
+    int ia = 0, ib = 0, iu = 0;
+    uint32_t m = wu;
+    while (m) {
+      const int bit = __ffs(m) - 1;
+      m &= m - 1;
+      const int blk = 32 * k + bit;
+      const uint32_t inA = (wa >> bit) & 1u, inB = (wb >> bit) & 1u;
+      if (write_rows) {
+        if (inA) col_idx[baseA + runA + oa + ia++] = blk;
+        if (inB) col_idx[baseB + runB + ob + ib++] = blk;
+      }
+      tile_col[baseT + runT + ou + iu++] = (blk << 2) | static_cast<int>(inA) | (static_cast<int>(inB) << 1);
+    }
+    runA += totA;
+    runB += totB;
+    runT += totU;
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// Tiles from a caller-made CSR
+// ---------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) csr_to_bits_kernel(const int32_t* __restrict__ row_ptr,
+                                                          const int32_t* __restrict__ col_idx, int64_t rows,
+                                                          int nB, int nWords, uint32_t* bits, int32_t* dev_status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  for (int k = lane; k < nWords; k += 32) bits[r * nWords + k] = 0u;
+  __syncwarp();
+  const int32_t lo = row_ptr[r], hi = row_ptr[r + 1];
+  for (int32_t i = lo + lane; i < hi; i += 32) {
+    const int32_t c = col_idx[i];
+    if (c < 0 || c >= nB) {
+      report(dev_status, FVA_DEVERR_BAD_LIST);
+      continue;
+    }
+    atomicOr(&bits[r * nWords + (c >> 5)], 1u << (c & 31));
+  }
+}
+
+__global__ void __launch_bounds__(256) tile_cost_kernel(const uint32_t* __restrict__ bits, int nB, int nWords,
+                                                        int nPairs, int64_t tiles, int32_t* tile_cost) {
+  const int lane = threadIdx.x & 31;
+  const int64_t tile = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (tile >= tiles) return;
+  const int64_t bh = tile / nPairs;
+  const int t = static_cast<int>(tile - bh * nPairs);
+  const int64_t rA = bh * nB + 2 * t;
+  const bool hasB = 2 * t + 1 < nB;
+  int u = 0;
+  for (int k = lane; k < nWords; k += 32)
+    u += __popc(bits[rA * nWords + k] | (hasB ? bits[(rA + 1) * nWords + k] : 0u));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+  if (lane == 0) tile_cost[tile] = u;
+}
+
+// ---------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------
+static int select_rows_per_cta(const Dims& D) {
+  const size_t arena = warp_arena_bytes(static_cast<int>(D.nB), static_cast<int>(D.nWords));
+  int r = 8;
+  while (r > 2 && arena * r > 200 * 1024) r -= 2;
+  return (arena * r > 200 * 1024) ? 0 : r;
+}
+
+static cudaError_t launch_order_and_emit(const Dims& D, const fva_mask* m, int order, const RouteScratch& ws,
+                                         int write_rows, cudaStream_t st) {
+  if (order == FVA_ORDER_NATURAL) {
+    int grid = static_cast<int>((D.tiles + 255) / 256);
+    order_natural_kernel<<<grid, 256, 0, st>>>(m->worklist, D.tiles);
+  } else if (order == FVA_ORDER_LPT) {
+    order_lpt_kernel<<<static_cast<int>((D.tiles + 255) / 256), 256, 0, st>>>(m->tile_cost, D.tiles, m->worklist);
+  } else {
+    const size_t smem = static_cast<size_t>(D.nPairs) * 4;
+    cudaFuncSetAttribute(order_head_lpt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    order_head_lpt_kernel<<<static_cast<int>(D.BH), 256, smem, st>>>(m->tile_cost, ws.head_load,
+                                                                     static_cast<int>(D.BH),
+                                                                     static_cast<int>(D.nPairs), m->worklist);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  emit_kernel<<<static_cast<int>((D.tiles + 7) / 8), 256, 0, st>>>(
+      ws.bits, static_cast<int>(D.nB), static_cast<int>(D.nWords), static_cast<int>(D.nPairs), D.tiles,
+      m->row_ptr, m->tile_ptr, m->col_idx, m->tile_col, write_rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route(const Dims& D, const double* pq, const double* pk, double p, int k_floor, int order,
+                         const fva_mask* m, const RouteScratch& ws, int32_t* dev_status, cudaStream_t st) {
+  const int nB = static_cast<int>(D.nB);
+  {
+    const dim3 grid((nB + kST - 1) / kST, (nB + kST - 1) / kST, static_cast<unsigned>(D.BH));
+    route_scores_kernel<<<grid, 256, 0, st>>>(pq, pk, ws.scores, nB, static_cast<int>(D.d),
+                                              sqrt(static_cast<double>(D.d)));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  {
+    const int rpc = select_rows_per_cta(D);
+    const size_t smem = warp_arena_bytes(nB, static_cast<int>(D.nWords)) * rpc;
+    cudaFuncSetAttribute(route_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    const dim3 grid((nB + rpc - 1) / rpc, static_cast<unsigned>(D.BH));
+    route_select_kernel<<<grid, 32 * rpc, smem, st>>>(ws.scores, nB, static_cast<int>(D.nWords),
+                                                     static_cast<int>(D.nPairs), p, k_floor, ws.bits, ws.row_cnt,
+                                                     m->tile_cost, dev_status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  finish_kernel<<<1, 1024, 0, st>>>(ws.row_cnt, D.rows, m->tile_cost, D.tiles, nB, static_cast<int>(D.nPairs),
+                                    static_cast<int>(D.BH), m->row_ptr, m->tile_ptr, m->head_kept, ws.head_load,
+                                    m->capacity, m->tile_capacity, dev_status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_order_and_emit(D, m, order, ws, 1, st);
+}
+
+cudaError_t launch_build_tiles(const Dims& D, const fva_mask* m, int order, const RouteScratch& ws,
+                               int32_t* dev_status, cudaStream_t st) {
+  csr_to_bits_kernel<<<static_cast<int>((D.rows + 7) / 8), 256, 0, st>>>(
+      m->row_ptr, m->col_idx, D.rows, static_cast<int>(D.nB), static_cast<int>(D.nWords), ws.bits, dev_status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  tile_cost_kernel<<<static_cast<int>((D.tiles + 7) / 8), 256, 0, st>>>(
+      ws.bits, static_cast<int>(D.nB), static_cast<int>(D.nWords), static_cast<int>(D.nPairs), D.tiles, m->tile_cost);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  finish_kernel<<<1, 1024, 0, st>>>(nullptr, D.rows, m->tile_cost, D.tiles, static_cast<int>(D.nB),
+                                    static_cast<int>(D.nPairs), static_cast<int>(D.BH), m->row_ptr, m->tile_ptr,
+                                    m->head_kept, ws.head_load, m->capacity, m->tile_capacity, dev_status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_order_and_emit(D, m, order, ws, 0, st);
+}
+
+bool route_shape_supported(const Dims& D) { return select_rows_per_cta(D) > 0; }
+
+}  // namespace fva

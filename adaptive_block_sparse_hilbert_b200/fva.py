@@ -1,0 +1,228 @@
+"""Thin ctypes binding of libfva (argument marshalling only).
+
+Every function here forwards to the C entry point of the same name in libfva.so; all
+compute runs in the library's sm_100a kernels. Tensors are torch CUDA tensors (device
+memory and streams are the only things PyTorch provides). Importing this module loads
+libfva.so and raises if it is missing: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfva.so")
+
+FVA_OK = 0
+FVA_ERR_INVALID_ARG = -1
+FVA_ERR_UNSUPPORTED_SHAPE = -2
+FVA_ERR_CAPACITY = -3
+FVA_ERR_CUDA = -4
+FVA_ERR_DEVICE_TIMEOUT = -5
+FVA_ERR_WORKSPACE = -6
+FVA_ERR_ALIGNMENT = -7
+
+FVA_DEVERR_NONE = 0
+FVA_DEVERR_TIMEOUT = 1
+FVA_DEVERR_MASK = 2
+FVA_DEVERR_BAD_LIST = 3
+
+FVA_F32 = 0
+FVA_BF16 = 1
+FVA_FWD = 0
+FVA_INV = 1
+FVA_ORDER_NATURAL = 0
+FVA_ORDER_LPT = 1
+FVA_ORDER_HEAD_LPT = 2
+
+BLOCK = 64
+
+
+class fva_shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("T", ctypes.c_int32), ("Hg", ctypes.c_int32), ("Wg", ctypes.c_int32),
+                ("block", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class fva_mask(ctypes.Structure):
+    _fields_ = [("row_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p), ("capacity", ctypes.c_int64),
+                ("head_kept", ctypes.c_void_p), ("tile_ptr", ctypes.c_void_p), ("tile_col", ctypes.c_void_p),
+                ("tile_capacity", ctypes.c_int64), ("tile_cost", ctypes.c_void_p), ("worklist", ctypes.c_void_p)]
+
+
+class FvaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libfva.so not built at {LIB_PATH}; run python -m adaptive_block_sparse_hilbert_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    S = ctypes.POINTER(fva_shape)
+    M = ctypes.POINTER(fva_mask)
+    i32, i64, sz, dbl, flt = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_double, ctypes.c_float
+    sig = {
+        "fva_status_string": (ctypes.c_char_p, [i32]),
+        "fva_version": (i32, []),
+        "fva_num_tokens": (i64, [S]),
+        "fva_num_blocks": (i64, [S]),
+        "fva_num_tiles": (i64, [S]),
+        "fva_mask_capacity": (i64, [S]),
+        "fva_tile_capacity": (i64, [S]),
+        "fva_route_workspace_bytes": (sz, [S, i32]),
+        "fva_tiles_workspace_bytes": (sz, [S]),
+        "fva_hilbert_perm": (i32, [S, P, P, P]),
+        "fva_reorder": (i32, [S, P, P, P, P, i32, P]),
+        "fva_pool": (i32, [S, P, P, P]),
+        "fva_route": (i32, [S, P, P, P, P, dbl, i32, i32, M, P, sz, P, P]),
+        "fva_build_tiles": (i32, [S, M, i32, P, sz, P, P]),
+        "fva_sparse_attn": (i32, [S, P, P, P, M, P, flt, P, P]),
+        "fva_dense_attn": (i32, [S, P, P, P, P, flt, P, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+_lib = _load()
+EXPORTED = (
+    "fva_status_string", "fva_version", "fva_num_tokens", "fva_num_blocks", "fva_num_tiles", "fva_mask_capacity",
+    "fva_tile_capacity", "fva_route_workspace_bytes", "fva_tiles_workspace_bytes", "fva_hilbert_perm", "fva_reorder",
+    "fva_pool", "fva_route", "fva_build_tiles", "fva_sparse_attn", "fva_dense_attn",
+)
+
+
+def lib():
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return _lib.fva_status_string(int(status)).decode()
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn, rc):
+    if rc != FVA_OK:
+        raise FvaError(fn, rc)
+
+
+# ------------------------------------------------------------------------------ shapes
+
+def make_shape(B, H, d, T, Hg, Wg, dtype="bf16") -> fva_shape:
+    dt = {"bf16": FVA_BF16, "f32": FVA_F32, FVA_BF16: FVA_BF16, FVA_F32: FVA_F32}[dtype]
+    return fva_shape(B, H, d, T, Hg, Wg, BLOCK, dt)
+
+
+def fva_num_tokens(s): return _lib.fva_num_tokens(ctypes.byref(s))
+def fva_num_blocks(s): return _lib.fva_num_blocks(ctypes.byref(s))
+def fva_num_tiles(s): return _lib.fva_num_tiles(ctypes.byref(s))
+def fva_mask_capacity(s): return _lib.fva_mask_capacity(ctypes.byref(s))
+def fva_tile_capacity(s): return _lib.fva_tile_capacity(ctypes.byref(s))
+def fva_route_workspace_bytes(s, need_pool=False): return _lib.fva_route_workspace_bytes(ctypes.byref(s), int(need_pool))
+def fva_tiles_workspace_bytes(s): return _lib.fva_tiles_workspace_bytes(ctypes.byref(s))
+
+
+# ------------------------------------------------------------------------------ masks
+
+@dataclasses.dataclass
+class Mask:
+    """Device buffers of one block mask (owned by torch; passed to libfva as fva_mask)."""
+
+    row_ptr: torch.Tensor
+    col_idx: torch.Tensor
+    head_kept: torch.Tensor
+    tile_ptr: torch.Tensor
+    tile_col: torch.Tensor
+    tile_cost: torch.Tensor
+    worklist: torch.Tensor
+
+    @staticmethod
+    def allocate(s: fva_shape, device="cuda") -> "Mask":
+        B, H = s.B, s.H
+        nB = fva_num_blocks(s)
+        tiles = fva_num_tiles(s)
+        i32 = dict(dtype=torch.int32, device=device)
+        return Mask(
+            row_ptr=torch.empty(B * H * nB + 1, **i32),
+            col_idx=torch.empty(fva_mask_capacity(s), **i32),
+            head_kept=torch.empty(B * H, dtype=torch.int64, device=device),
+            tile_ptr=torch.empty(tiles + 1, **i32),
+            tile_col=torch.empty(fva_tile_capacity(s), **i32),
+            tile_cost=torch.empty(tiles, **i32),
+            worklist=torch.empty(tiles, **i32),
+        )
+
+    def c(self) -> fva_mask:
+        return fva_mask(self.row_ptr.data_ptr(), self.col_idx.data_ptr(), self.col_idx.numel(),
+                        self.head_kept.data_ptr(), self.tile_ptr.data_ptr(), self.tile_col.data_ptr(),
+                        self.tile_col.numel(), self.tile_cost.data_ptr(), self.worklist.data_ptr())
+
+
+# ------------------------------------------------------------------------------ entry points
+
+def fva_hilbert_perm(s, perm, inv, stream=None):
+    _check("fva_hilbert_perm", _lib.fva_hilbert_perm(ctypes.byref(s), _ptr(perm), _ptr(inv), _stream(stream)))
+
+
+def fva_reorder(s, x_in, x_out, pooled, perm, direction=FVA_FWD, stream=None):
+    _check("fva_reorder", _lib.fva_reorder(ctypes.byref(s), _ptr(x_in), _ptr(x_out), _ptr(pooled), _ptr(perm),
+                                           int(direction), _stream(stream)))
+
+
+def fva_pool(s, x_bhnd, pooled, stream=None):
+    _check("fva_pool", _lib.fva_pool(ctypes.byref(s), _ptr(x_bhnd), _ptr(pooled), _stream(stream)))
+
+
+def fva_route(s, q, k, pooled_q, pooled_k, p, k_floor, mask: Mask, workspace, order=FVA_ORDER_HEAD_LPT,
+              dev_status=None, stream=None):
+    m = mask.c() if isinstance(mask, Mask) else mask
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check("fva_route", _lib.fva_route(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(pooled_q), _ptr(pooled_k), float(p),
+                                       int(k_floor), int(order), ctypes.byref(m), _ptr(workspace), ws_bytes,
+                                       _ptr(dev_status), _stream(stream)))
+
+
+def fva_build_tiles(s, mask: Mask, workspace, order=FVA_ORDER_HEAD_LPT, dev_status=None, stream=None):
+    m = mask.c() if isinstance(mask, Mask) else mask
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check("fva_build_tiles", _lib.fva_build_tiles(ctypes.byref(s), ctypes.byref(m), int(order), _ptr(workspace),
+                                                   ws_bytes, _ptr(dev_status), _stream(stream)))
+
+
+def fva_sparse_attn(s, q, k, v, mask: Mask, o, scale=0.0, dev_status=None, stream=None):
+    m = mask.c() if isinstance(mask, Mask) else mask
+    _check("fva_sparse_attn", _lib.fva_sparse_attn(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(m),
+                                                   _ptr(o), float(scale), _ptr(dev_status), _stream(stream)))
+
+
+def fva_dense_attn(s, q, k, v, o, scale=0.0, dev_status=None, stream=None):
+    _check("fva_dense_attn", _lib.fva_dense_attn(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(o), float(scale),
+                                                 _ptr(dev_status), _stream(stream)))
+
+
+def call_raw(name, *args):
+    """Call an entry point and return its status instead of raising (for error-path tests)."""
+    return getattr(_lib, name)(*args)

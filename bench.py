@@ -1,0 +1,466 @@
+"""Benchmark: one attention layer of the FVAttn hot path on B200 through libfva.
+
+A step = Hilbert reorder of Q, K, V (+ fused pooling of Q and K) -> Top-p / Top-k_floor
+routing (scores, selection, CSR, tiles, work list) -> block-sparse attention -> inverse
+reorder of O, on one synthetic layer already resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--p 0.9]
+    python bench.py --impl reference ...      # the float64 oracle on the host cores
+
+Prints one JSON line (rank 0). The metric is milliseconds per attention layer (lower is
+better) with the attention kernel's kept-block TFLOPS against the measured bf16 peak.
+With N > 1 (torchrun) every rank runs its own replica of the layer on its own GPU (the
+path has no exchange step); `value` is then max-over-ranks time per step divided by the
+layers all ranks processed in it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from adaptive_block_sparse_hilbert_b200 import synth  # noqa: E402
+
+METRIC = "sparse attn ms/layer & kept-block TFLOPS vs B200 bf16 peak at 75.6k tokens"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LAUNCHES_PER_STEP = 10  # 3 forward reorders, 5 routing kernels, 1 attention, 1 inverse reorder
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+# ----------------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------------- schedule model
+
+def list_schedule(costs: np.ndarray, order: np.ndarray, slots: int):
+    """Greedy list scheduling (each free slot takes the next tile): per-slot loads."""
+    import heapq
+    heap = [(0, i) for i in range(slots)]
+    load = np.zeros(slots, dtype=np.int64)
+    for t in order:
+        l, i = heapq.heappop(heap)
+        load[i] = l + int(costs[t])
+        heapq.heappush(heap, (load[i], i))
+    return load
+
+
+def imbalance(costs: np.ndarray, BH: int, n_pairs: int, slots: int):
+    out = {}
+    ids = np.arange(costs.size)
+    orders = {
+        "natural": ids,
+        "lpt": np.lexsort((ids, -costs)),
+    }
+    load = costs.reshape(BH, n_pairs).sum(axis=1)
+    heads = np.lexsort((np.arange(BH), -load))
+    orders["head_lpt"] = np.concatenate([bh * n_pairs + np.lexsort((np.arange(n_pairs), -costs[bh * n_pairs:(bh + 1) * n_pairs]))
+                                         for bh in heads])
+    for k, o in orders.items():
+        l = list_schedule(costs, o, slots)
+        out[k] = {"max_over_mean": round(float(l.max() / l.mean()), 4),
+                  "max_over_min": round(float(l.max() / max(l.min(), 1)), 4)}
+    return out
+
+
+# ----------------------------------------------------------------------------------- oracle timing
+
+def oracle_sample(wl, L, n_heads: int, rows_per_head: int, seed: int = 0):
+    """Time the float64 oracle on a bounded sample and extrapolate to a full layer (ms)."""
+    import oracle as O
+    rng = np.random.default_rng(seed)
+    heads = rng.choice(wl.H, size=min(n_heads, wl.H), replace=False)
+    t0 = time.perf_counter()
+    perm, _ = O.hilbert_perm(wl.T, wl.Hg, wl.Wg)
+    t_perm = time.perf_counter() - t0
+    t_reorder = t_route = t_attn = 0.0
+    n_rows = 0
+    for h in heads:
+        t0 = time.perf_counter()
+        q = O.reorder(L.q[:, :, h:h + 1], perm)
+        k = O.reorder(L.k[:, :, h:h + 1], perm)
+        v = O.reorder(L.v[:, :, h:h + 1], perm)
+        t1 = time.perf_counter()
+        R = O.route(O.block_mean_pool(q), O.block_mean_pool(k), wl.d, wl.p, wl.k_floor)
+        t2 = time.perf_counter()
+        rows = [(0, 0, int(a)) for a in rng.choice(wl.nB, size=min(rows_per_head, wl.nB), replace=False)]
+        O.block_sparse_attention(q, k, v, R["row_ptr"], R["col_idx"], rows=rows)
+        t3 = time.perf_counter()
+        t_reorder += t1 - t0
+        t_route += t2 - t1
+        t_attn += t3 - t2
+        n_rows += len(rows)
+    nh = len(heads)
+    ms = 1e3 * (t_perm + (t_reorder + t_route) * wl.H / nh + t_attn * (wl.H * wl.nB) / n_rows)
+    sample = (f"{nh} of {wl.H} heads: reorder + pooling + full routing of each sampled head, attention on "
+              f"{rows_per_head} seeded query blocks per sampled head; time extrapolated linearly to all heads "
+              f"and all {wl.nB} query blocks (extrapolated)")
+    wall = t_perm + t_reorder + t_route + t_attn
+    return ms, sample, wall
+
+
+def cpu_cores():
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    threads = n
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            threads = max(int(i.get("num_threads", 1)) for i in info)
+    except Exception:
+        pass
+    return n, threads
+
+
+# ----------------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    wl = synth.WORKLOADS[args.workload]
+    wl = synth.Workload(**{**wl.__dict__, "p": args.p if args.p is not None else wl.p})
+    L = synth.make_layer(wl)
+    vals = []
+    sample = ""
+    for i in range(args.warmup + args.steps):
+        ms, sample, _ = oracle_sample(wl, L, n_heads=1, rows_per_head=8, seed=i)
+        if i >= args.warmup:
+            vals.append(ms)
+    cores, threads = cpu_cores()
+    v = float(np.median(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "ms/layer", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 3), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "tokens": wl.N, "heads": wl.H, "head_dim": wl.d, "p": wl.p,
+                   "k_floor": wl.k_floor, "block": 64},
+        "cpu_baseline": {"value": round(v, 3), "unit": "ms/layer", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(v, 3), "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------------- GPU arm
+
+def traffic_record(kernel_src: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it matches the source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+    r = rec.get("attn_bf16_kernel")
+    if not r or r.get("source_sha256") != sha:
+        return None
+    return r
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from adaptive_block_sparse_hilbert_b200 import fva, pipeline
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    wl = synth.WORKLOADS[args.workload]
+    if args.p is not None:
+        wl = synth.Workload(**{**wl.__dict__, "p": args.p})
+    L = synth.make_layer(wl)
+    s = fva.make_shape(wl.B, wl.H, wl.d, wl.T, wl.Hg, wl.Wg, wl.dtype)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+
+    def host(vals, bits):
+        if bits is not None:
+            return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        return torch.from_numpy(np.ascontiguousarray(vals)).pin_memory()
+
+    hq, hk, hv = host(L.q, L.q_bits), host(L.k, L.k_bits), host(L.v, L.v_bits)
+    ho = torch.empty_like(hq).pin_memory()
+    q, k, v = hq.to(dev), hk.to(dev), hv.to(dev)
+    o = torch.empty_like(q)
+    layer = pipeline.SparseAttentionLayer(s, wl.p, wl.k_floor, device=dev)
+    stream = torch.cuda.current_stream()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def step(marks=None):
+        if marks is not None:
+            marks[0].record(stream)
+        layer.reorder_inputs(q, k, v)
+        if marks is not None:
+            marks[1].record(stream)
+        layer.route()
+        if marks is not None:
+            marks[2].record(stream)
+        layer.attend()
+        if marks is not None:
+            marks[3].record(stream)
+        layer.restore_output(o)
+        if marks is not None:
+            marks[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    clocks = ClockSampler(local if world > 1 else torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    marks = [[ev() for _ in range(5)] for _ in range(args.steps)]
+    start, end = ev(), ev()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    start.record(stream)
+    for i in range(args.steps):
+        step(marks[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    total_ms = start.elapsed_time(end)
+    clk = clocks.stop()
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+        total_ms = float(t.item())
+    status = int(layer.dev_status.item())
+
+    stage = np.array([[m[j].elapsed_time(m[j + 1]) for j in range(4)] for m in marks])
+    t_reorder, t_route, t_attn, t_inv = [float(np.mean(stage[:, j])) for j in range(4)]
+    ms_step = total_ms / args.steps
+
+    # mask statistics and algorithmic work
+    rp = layer.mask.row_ptr.cpu().numpy().astype(np.int64)
+    nB, N, d, BH = wl.nB, wl.N, wl.d, wl.B * wl.H
+    kept = int(rp[-1])
+    sizes = np.minimum(64, N - 64 * np.arange(nB)).astype(np.int64)
+    ci = layer.mask.col_idx[:kept].cpu().numpy().astype(np.int64)
+    counts = np.diff(rp)
+    a_idx = np.repeat(np.arange(BH * nB) % nB, counts)
+    kept_flops = float(4 * d * np.sum(sizes[a_idx] * sizes[ci]))
+    costs = layer.mask.tile_cost.cpu().numpy().astype(np.int64)
+    issued_flops = float(4 * d * 128 * 64 * costs.sum())
+    dense_flops = float(4 * d * BH * N * N)
+    reorder_bytes = float(6 * wl.B * N * wl.H * d * (2 if wl.dtype == "bf16" else 4) + 2 * BH * nB * d * 8)
+
+    pk, how = peaks()
+    peak_tf = float(pk.get("bf16_tflops_sustained", pk.get("bf16_tflops")))
+    hbm = float(pk["hbm_gbs"])
+    achieved_tf = kept_flops / (t_attn * 1e-3) / 1e12
+    tr = traffic_record(os.path.join(ROOT, "adaptive_block_sparse_hilbert_b200", "csrc", "attn_tc.cu"))
+    traffic = None
+    if tr and tr.get("workload") == wl.name:
+        traffic = tr.get("traffic_bytes_per_launch")
+
+    # dense density-1 reference kernel (same launch family), timed separately
+    dense_ms = None
+    if not args.no_dense:
+        od = torch.empty_like(layer.qh)
+        for _ in range(2):
+            fva.fva_dense_attn(s, layer.qh, layer.kh, layer.vh, od, 0.0, layer.dev_status)
+        e0, e1 = ev(), ev()
+        e0.record(stream)
+        for _ in range(3):
+            fva.fva_dense_attn(s, layer.qh, layer.kh, layer.vh, od, 0.0, layer.dev_status)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = e0.elapsed_time(e1) / 3
+        del od
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    h2d = 3 * hq.numel() * hq.element_size()
+    d2h = ho.numel() * ho.element_size()
+    for _ in range(2):
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+        layer.forward(q, k, v, o)
+        ho.copy_(o, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    n_e2e = max(3, min(args.steps, 10))
+    e0.record(stream)
+    for _ in range(n_e2e):
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+        layer.forward(q, k, v, o)
+        ho.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+    imb = imbalance(costs, BH, (nB + 1) // 2, 2 * sm_count)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores, threads = cpu_cores()
+        ms_cpu, sample, wall = oracle_sample(wl, L, n_heads=args.cpu_heads, rows_per_head=args.cpu_rows)
+        cpu = {"value": round(ms_cpu, 1), "unit": "ms/layer", "cores": threads, "kind": "oracle", "sample": sample,
+               "wall_s": round(wall, 1), "affinity_cores": cores}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": round(ms_step / world, 4),
+            "unit": "ms/layer",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 4),
+            "higher_is_better": False,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "tokens": N, "grid": [wl.T, wl.Hg, wl.Wg], "heads": wl.H,
+                       "head_dim": d, "block": 64, "p": wl.p, "k_floor": wl.k_floor, "order": "head_lpt",
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (3 x %.0f MB)" % (q.numel() * q.element_size() / 1e6)},
+            "kept_tflops": round(achieved_tf, 1),
+            "kept_tflops_frac_of_peak": round(achieved_tf / peak_tf, 4),
+            "issued_tflops": round(issued_flops / (t_attn * 1e-3) / 1e12, 1),
+            "density": round(kept / (BH * nB * nB), 4),
+            "stage_ms": {"reorder_qkv": round(t_reorder, 4), "route": round(t_route, 4), "attn": round(t_attn, 4),
+                         "inverse_o": round(t_inv, 4)},
+            "dense_attn_ms": round(dense_ms, 3) if dense_ms else None,
+            "dense_attn_tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 1) if dense_ms else None,
+            "reorder_gbs": round(reorder_bytes / (t_reorder * 1e-3) / 1e9, 1),
+            "reorder_hbm_frac": round(reorder_bytes / (t_reorder * 1e-3) / 1e9 / hbm, 4),
+            "roofline": {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": round(achieved_tf / peak_tf, 4), "traffic": traffic,
+                         "kernel": "attn_bf16_kernel (fva_sparse_attn)",
+                         "peak_source": f"{how} bf16_tflops_sustained (kernel timed inside a multi-second loop)"},
+            "imbalance_sm_slots": imb,
+            "e2e": {"value": round(e2e_ms, 3), "unit": "ms/layer", "h2d_bytes_per_step": int(h2d),
+                    "d2h_bytes_per_step": int(d2h)},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clk,
+            "dev_status": status,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0 if status == 0 else 3
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--p", type=float, default=None)
+    ap.add_argument("--impl", default="fva", choices=["fva", "reference"])
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-heads", type=int, default=2)
+    ap.add_argument("--cpu-rows", type=int, default=24)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        sys.exit(run_reference(args))
+    sys.exit(run_gpu(args))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,206 @@
+/*
+ * fva.h -- C ABI of libfva: Hilbert-ordered block routing and block-sparse attention
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the FVAttn pages (arXiv 2607.16190):
+ *   [aixai] aixai.ru FVAttn blog -- "Sparse-routing frontend", "Top-p vs Top-k",
+ *           "Runtime Load Balancing (RLB)", sparse-attention section;
+ *   [PD]    longzhangge.com PaperDaily FVAttn article -- 方法揭秘 (method), 龙迷三问 (Q&A);
+ *   [abs]   mlsanity.com "FVAttn: Adaptive Sparse Attention with Runtime Load Balancing
+ *           for Video Generation" -- abstract.
+ *
+ * Conventions (all entry points):
+ *   - Every function returns an int status: FVA_OK (0) or a negative FVA_ERR_* code.
+ *     fva_status_string() gives its text. No exception crosses the ABI.
+ *   - The caller owns all memory. Pointers named *_dev are device pointers (cudaMalloc /
+ *     torch CUDA tensors), 16-byte aligned unless stated otherwise. The library allocates
+ *     no device memory; scratch space is passed in as a caller-owned workspace.
+ *   - Work is enqueued asynchronously on the given stream (NULL = legacy default
+ *     stream); outputs are valid after the stream is synchronised.
+ *   - Host-detectable errors (null pointers, unsupported shapes, capacity or workspace
+ *     too small, p outside (0, 1], negative k_floor) return before anything is
+ *     enqueued. Errors found on the device (a bounded wait that ran out, an
+ *     inconsistent mask) are written to the optional caller-provided int32 dev_status
+ *     (device memory, expected to hold 0 on entry; set to a nonzero FVA_DEVERR_* code)
+ *     and leave the device usable.
+ *   - Layouts: x_bnhd = [B, N, H, d] raster token order (n = t*Hg*Wg + y*Wg + x);
+ *     x_bhnd = [B, H, N, d] Hilbert order; pooled = [B, H, nB, d] float64.
+ *   - Sizes: N = T*Hg*Wg, block = 64, nB = ceil(N / 64), nPairs = ceil(nB / 2);
+ *     a "row" is one (b, h, query block a), r = (b*H + h)*nB + a; a "tile" is a pair
+ *     of adjacent query blocks (2t, 2t+1) of one (b, h), id = (b*H + h)*nPairs + t.
+ */
+#ifndef FVA_H_
+#define FVA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FVA_API __attribute__((visibility("default")))
+#else
+#define FVA_API
+#endif
+
+typedef struct CUstream_st* fva_stream_t; /* identical to cudaStream_t */
+
+enum {
+  FVA_OK = 0,
+  FVA_ERR_INVALID_ARG = -1,       /* null pointer, bad enum, p or k_floor out of range */
+  FVA_ERR_UNSUPPORTED_SHAPE = -2, /* shape/dtype combination this build does not handle */
+  FVA_ERR_CAPACITY = -3,          /* mask buffers smaller than fva_mask_capacity() etc. */
+  FVA_ERR_CUDA = -4,              /* a CUDA runtime/driver call failed */
+  FVA_ERR_DEVICE_TIMEOUT = -5,    /* reported through dev_status only */
+  FVA_ERR_WORKSPACE = -6,         /* workspace smaller than the query function says */
+  FVA_ERR_ALIGNMENT = -7          /* a device pointer is not 16-byte aligned */
+};
+
+/* Codes written to dev_status by kernels. */
+enum {
+  FVA_DEVERR_NONE = 0,
+  FVA_DEVERR_TIMEOUT = 1,   /* an mbarrier wait in the attention kernel ran out (~2 s) */
+  FVA_DEVERR_MASK = 2,      /* a routed row's kept count disagreed with max(L_p, L_k) */
+  FVA_DEVERR_BAD_LIST = 3   /* a tile list entry was out of range */
+};
+
+enum { FVA_F32 = 0, FVA_BF16 = 1 };
+enum { FVA_FWD = 0, FVA_INV = 1 };
+/* Order of the attention work list (tiles are launched in this order). */
+enum {
+  FVA_ORDER_NATURAL = 0,    /* tile id order */
+  FVA_ORDER_LPT = 1,        /* longest first over all tiles (cost desc, id asc) */
+  FVA_ORDER_HEAD_LPT = 2    /* heads by total cost desc (id asc), longest first inside a head */
+};
+
+/* Problem shape. block must be 64. dtype is FVA_F32 or FVA_BF16. */
+typedef struct fva_shape {
+  int32_t B, H, d;
+  int32_t T, Hg, Wg;
+  int32_t block;
+  int32_t dtype;
+} fva_shape;
+
+/* Block mask in CSR form plus the tile-level lists the attention kernel reads.
+ * All pointers are device pointers owned by the caller.
+ *   row_ptr   int32 [B*H*nB + 1]       CSR offsets over rows r
+ *   col_idx   int32 [capacity]         kept key blocks of each row, ascending
+ *   head_kept int64 [B*H]              kept (query block, key block) pairs per head:
+ *                                      the head's load L_h ([aixai] RLB section)
+ *   tile_ptr  int32 [B*H*nPairs + 1]   offsets into tile_col
+ *   tile_col  int32 [tile_capacity]    union of the two rows' lists, ascending; entry =
+ *                                      key_block*4 | (row 2t keeps it) | (row 2t+1 keeps it)<<1
+ *   tile_cost int32 [B*H*nPairs]       number of entries of each tile (its work)
+ *   worklist  int32 [B*H*nPairs]       tile ids in launch order (see FVA_ORDER_*)
+ */
+typedef struct fva_mask {
+  int32_t* row_ptr;
+  int32_t* col_idx;
+  int64_t capacity;
+  int64_t* head_kept;
+  int32_t* tile_ptr;
+  int32_t* tile_col;
+  int64_t tile_capacity;
+  int32_t* tile_cost;
+  int32_t* worklist;
+} fva_mask;
+
+FVA_API const char* fva_status_string(int status);
+FVA_API int fva_version(void);
+
+/* Derived sizes; -1 for an invalid shape. */
+FVA_API int64_t fva_num_tokens(const fva_shape* s);
+FVA_API int64_t fva_num_blocks(const fva_shape* s);
+FVA_API int64_t fva_num_tiles(const fva_shape* s);
+/* Entries col_idx / tile_col must hold: B*H*nB*nB and B*H*nPairs*nB. */
+FVA_API int64_t fva_mask_capacity(const fva_shape* s);
+FVA_API int64_t fva_tile_capacity(const fva_shape* s);
+/* Bytes of workspace fva_route needs (with need_pool != 0: also room to pool Q and K). */
+FVA_API size_t fva_route_workspace_bytes(const fva_shape* s, int need_pool);
+
+/*
+ * Hilbert token order ("video-aware block organization": [aixai] "Sparse-routing
+ * frontend"; [PD] 方法揭秘). Per frame, the cells (y, x) are visited in the order of the
+ * 2-D Hilbert curve on the enclosing 2^m x 2^m square (m = ceil(log2(max(Hg, Wg))),
+ * out-of-grid cells skipped, first step (0,0) -> (x=0, y=1)); frames follow in t order.
+ * perm_dev[i] = raster index of the token at Hilbert position i; inv_dev = perm^-1.
+ * Both int32 [N], device memory.
+ */
+FVA_API int fva_hilbert_perm(const fva_shape* s, int32_t* perm_dev, int32_t* inv_dev, fva_stream_t stream);
+
+/*
+ * Token reorder with fused block mean-pooling ([aixai] "Sparse-routing frontend"; [PD]
+ * 方法揭秘: block importance from pooled Q/K).
+ *   FVA_FWD: x_out[b, h, i, :] = x_in[b, perm[i], h, :]   ([B,N,H,d] -> [B,H,N,d]);
+ *            if pooled_dev != NULL also pooled[b, h, a, :] = mean of x_out rows
+ *            [64a, min(64a+64, N)) in float64 (exact sum of the inputs, then / n_a).
+ *   FVA_INV: x_out[b, perm[i], h, :] = x_in[b, h, i, :]   ([B,H,N,d] -> [B,N,H,d]);
+ *            pooled_dev must be NULL.
+ * Element type from s->dtype; d * sizeof(elem) must be a multiple of 16 and <= 1024.
+ * x_in and x_out must not overlap.
+ */
+FVA_API int fva_reorder(const fva_shape* s, const void* x_in_dev, void* x_out_dev, double* pooled_dev,
+                const int32_t* perm_dev, int direction, fva_stream_t stream);
+
+/* Block mean-pool of an already Hilbert-ordered [B,H,N,d] tensor into float64 [B,H,nB,d]. */
+FVA_API int fva_pool(const fva_shape* s, const void* x_bhnd_dev, double* pooled_dev, fva_stream_t stream);
+
+/*
+ * Top-p routing with a Top-k safety floor ([aixai] "Top-p vs Top-k", "Sparse-routing
+ * frontend"; [PD] 方法揭秘, 龙迷三问). For every row (b, h, a):
+ *   s_ab = pooled_q[a] . pooled_k[b] / sqrt(d)          (float64)
+ *   P_ab = softmax_b(s_ab)                              (float64)
+ *   order key blocks by s descending, ties to the lower block index;
+ *   L_p  = length of the shortest prefix whose cumulative P reaches p (p = 1: all);
+ *   L    = max(L_p, min(k_floor, nB));  the first L blocks of the order are kept.
+ * Cumulative masses are summed exactly in 2^-52 fixed point, so a row's decision can
+ * differ from an exact float64 evaluation only when a cumulative mass lies within
+ * ~nB*2^-52 of p.
+ * Inputs: either pooled_q_dev/pooled_k_dev (float64 [B,H,nB,d], e.g. from fva_reorder)
+ * or, when both are NULL, q_bhnd_dev/k_bhnd_dev (Hilbert-ordered, pooled here into the
+ * workspace; needs fva_route_workspace_bytes(s, 1)).
+ * Outputs: every array of *mask (row_ptr, col_idx, head_kept, tile_ptr, tile_col,
+ * tile_cost, worklist); mask->capacity >= fva_mask_capacity(s) and
+ * mask->tile_capacity >= fva_tile_capacity(s) are required. order is a FVA_ORDER_*.
+ * 0 < p <= 1, k_floor >= 0.
+ */
+FVA_API int fva_route(const fva_shape* s, const void* q_bhnd_dev, const void* k_bhnd_dev,
+              const double* pooled_q_dev, const double* pooled_k_dev, double p, int k_floor,
+              int order, const fva_mask* mask, void* workspace_dev, size_t workspace_bytes,
+              int32_t* dev_status, fva_stream_t stream);
+
+/* Bytes of workspace fva_build_tiles needs. */
+FVA_API size_t fva_tiles_workspace_bytes(const fva_shape* s);
+
+/*
+ * Tile lists for a caller-made row-level CSR mask (mask->row_ptr / col_idx filled, each
+ * row ascending, unique, in [0, nB)). Fills tile_ptr, tile_col, tile_cost, worklist and
+ * head_kept the same way fva_route does.
+ */
+FVA_API int fva_build_tiles(const fva_shape* s, const fva_mask* mask, int order, void* workspace_dev,
+                    size_t workspace_bytes, int32_t* dev_status, fva_stream_t stream);
+
+/*
+ * Block-sparse attention ([aixai] sparse-attention section: only the kept key blocks of
+ * a query block are computed). For each query i in block a of (b, h):
+ *   o_i = sum_j softmax_j(scale * q_i . k_j) v_j  over the valid keys j of the kept blocks
+ * (no causal mask). q, k, v, o: [B,H,N,d] Hilbert order, dtype s->dtype (bf16: d in
+ * {64, 128}, fp32 accumulation, bf16 output; fp32: d % 4 == 0, d <= 128).
+ * scale <= 0 selects 1/sqrt(d). Reads mask->tile_ptr, tile_col, worklist (bf16) or
+ * mask->row_ptr, col_idx (fp32). o must not overlap q, k or v.
+ */
+FVA_API int fva_sparse_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev,
+                    const fva_mask* mask, void* o_dev, float scale, int32_t* dev_status,
+                    fva_stream_t stream);
+
+/* Dense attention (every block kept): the in-house density-1 reference. Same layouts. */
+FVA_API int fva_dense_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev,
+                   void* o_dev, float scale, int32_t* dev_status, fva_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FVA_H_ */

@@ -1,0 +1,105 @@
+"""The C ABI library loads and exports what include/fva.h declares; host-side checks
+(no device work is enqueued by any call here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from adaptive_block_sparse_hilbert_b200 import fva
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "fva.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FVA_API\s+[\w\s\*]*?\b(fva_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert len(names) >= 16
+    lib = ctypes.CDLL(fva.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(fva.EXPORTED)
+
+
+def test_no_internal_symbols_exported():
+    out = os.popen(f"nm -D --defined-only {fva.LIB_PATH}").read()
+    syms = [l.split()[-1] for l in out.splitlines() if " T " in l]
+    assert syms, out
+    assert all(s.startswith("fva_") or s.startswith("_init") or s.startswith("_fini") for s in syms), syms
+
+
+def test_status_strings():
+    assert fva.status_string(0) == "ok"
+    assert "capacity" in fva.status_string(fva.FVA_ERR_CAPACITY)
+    assert fva.status_string(-99) == "unknown status"
+
+
+@pytest.mark.parametrize("wid", [0, 1, 2, 3])
+def test_derived_sizes(wid):
+    from adaptive_block_sparse_hilbert_b200 import synth
+    wl = synth.WORKLOADS[wid]
+    s = fva.make_shape(wl.B, wl.H, wl.d, wl.T, wl.Hg, wl.Wg, wl.dtype)
+    N = wl.T * wl.Hg * wl.Wg
+    nB = (N + 63) // 64
+    assert fva.fva_num_tokens(s) == N
+    assert fva.fva_num_blocks(s) == nB
+    assert fva.fva_num_tiles(s) == wl.H * ((nB + 1) // 2)
+    assert fva.fva_mask_capacity(s) == wl.H * nB * nB
+    assert fva.fva_tile_capacity(s) == wl.H * ((nB + 1) // 2) * nB
+    ws0 = fva.fva_route_workspace_bytes(s, False)
+    ws1 = fva.fva_route_workspace_bytes(s, True)
+    assert ws0 >= wl.H * nB * nB * 8 and ws1 >= ws0 + 2 * wl.H * nB * wl.d * 8
+    assert 0 < fva.fva_tiles_workspace_bytes(s) < ws0
+
+
+def test_invalid_shapes_rejected():
+    bad = [
+        fva.make_shape(1, 2, 64, 0, 16, 16),       # T = 0
+        fva.make_shape(1, 2, 60, 4, 16, 16),       # d*2 not a multiple of 16
+        fva.fva_shape(1, 2, 64, 4, 16, 16, 32, fva.FVA_BF16),  # block != 64
+        fva.fva_shape(1, 2, 64, 4, 16, 16, 64, 7),  # bad dtype
+    ]
+    for s in bad:
+        assert fva.fva_num_tokens(s) == -1
+        assert fva.fva_route_workspace_bytes(s) == 0
+
+
+def test_host_validation_before_any_launch():
+    s = fva.make_shape(1, 2, 64, 4, 16, 16, "f32")
+    P = ctypes.c_void_p
+    one = P(16)  # a non-null dummy pointer; validation fails before it is ever used
+    rc = fva.call_raw("fva_reorder", ctypes.byref(s), None, one, None, one, 0, None)
+    assert rc == fva.FVA_ERR_INVALID_ARG
+    rc = fva.call_raw("fva_reorder", ctypes.byref(s), one, one, None, one, 5, None)
+    assert rc == fva.FVA_ERR_INVALID_ARG
+    rc = fva.call_raw("fva_reorder", ctypes.byref(s), one, P(48), P(64), one, fva.FVA_INV, None)
+    assert rc == fva.FVA_ERR_INVALID_ARG  # INV takes no pooled output
+    rc = fva.call_raw("fva_reorder", ctypes.byref(s), P(17), P(48), None, one, 0, None)
+    assert rc == fva.FVA_ERR_ALIGNMENT
+    m = fva.fva_mask(16, 16, 10, 16, 16, 16, 10, 16, 16)
+    # p out of range, negative floor, bad order, too-small capacity, too-small workspace
+    assert fva.call_raw("fva_route", ctypes.byref(s), one, one, None, None, 0.0, 2, 2, ctypes.byref(m), one, 1 << 30,
+                        None, None) == fva.FVA_ERR_INVALID_ARG
+    assert fva.call_raw("fva_route", ctypes.byref(s), one, one, None, None, 1.5, 2, 2, ctypes.byref(m), one, 1 << 30,
+                        None, None) == fva.FVA_ERR_INVALID_ARG
+    assert fva.call_raw("fva_route", ctypes.byref(s), one, one, None, None, float("nan"), 2, 2, ctypes.byref(m), one,
+                        1 << 30, None, None) == fva.FVA_ERR_INVALID_ARG
+    assert fva.call_raw("fva_route", ctypes.byref(s), one, one, None, None, 0.9, -1, 2, ctypes.byref(m), one, 1 << 30,
+                        None, None) == fva.FVA_ERR_INVALID_ARG
+    assert fva.call_raw("fva_route", ctypes.byref(s), one, one, None, None, 0.9, 2, 9, ctypes.byref(m), one, 1 << 30,
+                        None, None) == fva.FVA_ERR_INVALID_ARG
+    assert fva.call_raw("fva_route", ctypes.byref(s), one, one, None, None, 0.9, 2, 2, ctypes.byref(m), one, 1 << 30,
+                        None, None) == fva.FVA_ERR_CAPACITY
+    big = fva.fva_mask(16, 16, 1 << 20, 16, 16, 16, 1 << 20, 16, 16)
+    assert fva.call_raw("fva_route", ctypes.byref(s), one, one, None, None, 0.9, 2, 2, ctypes.byref(big), one, 64,
+                        None, None) == fva.FVA_ERR_WORKSPACE
+    # bf16 attention supports d in {64, 128} only
+    s96 = fva.make_shape(1, 2, 96, 4, 16, 16, "bf16")
+    assert fva.call_raw("fva_dense_attn", ctypes.byref(s96), one, one, one, P(4096), ctypes.c_float(0.0), None,
+                        None) == fva.FVA_ERR_UNSUPPORTED_SHAPE
+    assert fva.call_raw("fva_sparse_attn", ctypes.byref(s), one, one, one, None, P(4096), ctypes.c_float(0.0), None,
+                        None) == fva.FVA_ERR_INVALID_ARG

@@ -1,0 +1,188 @@
+"""GPU parity: block-sparse and dense attention (C ABI vs oracle).
+
+Tolerances: bf16 inputs max-abs 2e-2 and mean-abs 2e-3; fp32 inputs max-abs 1e-4. Both
+sides use the same (GPU-routed) mask, so outputs are compared on every row; the masks
+themselves are checked against the oracle in test_gpu_route.py.
+"""
+import numpy as np
+import pytest
+
+from adaptive_block_sparse_hilbert_b200 import synth
+import oracle as O
+from tests import _common as C
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_sparse(run):
+    import torch
+    run.layer.attend()
+    torch.cuda.synchronize()
+    assert run.status() == 0
+    return run.layer.oh.float().cpu().numpy().astype(np.float64)
+
+
+def _run_dense(run):
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import fva
+    o = torch.empty_like(run.layer.qh)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fva.fva_dense_attn(run.shape, run.layer.qh, run.layer.kh, run.layer.vh, o, 0.0, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    return o.float().cpu().numpy().astype(np.float64)
+
+
+def _tol(wl, got, want, what):
+    mx, mean = C.err_stats(got, want)
+    print(f"{wl.name} {what}: max-abs {mx:.3e} mean-abs {mean:.3e}")
+    if wl.dtype == "bf16":
+        assert mx <= C.BF16_MAX_ABS and mean <= C.BF16_MEAN_ABS, (mx, mean)
+    else:
+        assert mx <= C.F32_MAX_ABS, mx
+
+
+SMALL = [
+    synth.WORKLOADS[0],                                                  # fp32, 16 blocks
+    synth.custom_workload(3, 10, 13, 3, 64, "bf16", seed=31),            # nB = 7 (odd), tail of 6
+    synth.custom_workload(2, 9, 9, 2, 128, "bf16", seed=32),             # nB = 3, tail of 34
+    synth.custom_workload(4, 20, 20, 2, 128, "bf16", seed=33, tau=("logU", 2.0, 6.0)),  # sparse
+    synth.custom_workload(1, 8, 8, 1, 64, "bf16", seed=34),              # a single block
+    synth.custom_workload(2, 5, 7, 2, 64, "f32", seed=35),               # fp32 ragged
+    synth.custom_workload(5, 16, 16, 2, 128, "bf16", seed=36, p=0.7, k_floor=1),
+]
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_sparse_and_dense_small(wl):
+    L = synth.make_layer(wl)
+    run = C.GpuRun(wl, L)
+    g = run.mask_np()
+    perm, _ = O.hilbert_perm(wl.T, wl.Hg, wl.Wg)
+    qh, kh, vh = C.hilbert_bhnd(L, perm)
+    want = O.assemble(O.block_sparse_attention(qh, kh, vh, g["row_ptr"], g["col_idx"]), wl.B, wl.H, wl.N, wl.d)
+    _tol(wl, _run_sparse(run), want, "sparse")
+    _tol(wl, _run_dense(run), O.dense_attention(qh, kh, vh), "dense")
+
+
+def test_end_to_end_raster_output():
+    """forward(): reorder -> route -> attention -> inverse reorder equals the oracle in raster order."""
+    import torch
+    wl = synth.custom_workload(3, 10, 13, 3, 64, "bf16", seed=37)
+    L = synth.make_layer(wl)
+    run = C.GpuRun(wl, L)
+    out = torch.empty_like(run.q)
+    run.layer.forward(run.q, run.k, run.v, out)
+    torch.cuda.synchronize()
+    g = run.mask_np()
+    perm, _ = O.hilbert_perm(wl.T, wl.Hg, wl.Wg)
+    qh, kh, vh = C.hilbert_bhnd(L, perm)
+    want_h = O.assemble(O.block_sparse_attention(qh, kh, vh, g["row_ptr"], g["col_idx"]), wl.B, wl.H, wl.N, wl.d)
+    _tol(wl, out.float().cpu().numpy().astype(np.float64), O.inverse_reorder(want_h, perm), "forward")
+
+
+def _custom_mask_run(wl, lists_fn):
+    """Run the sparse kernel with a hand-made CSR mask (tiles built by fva_build_tiles)."""
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import fva
+    L = synth.make_layer(wl)
+    run = C.GpuRun(wl, L)
+    BH, nB = wl.B * wl.H, wl.nB
+    lists = [np.array(sorted(lists_fn(bh, a)), dtype=np.int32) for bh in range(BH) for a in range(nB)]
+    rp = np.concatenate([[0], np.cumsum([x.size for x in lists])]).astype(np.int32)
+    ci = np.concatenate(lists).astype(np.int32)
+    m = fva.Mask.allocate(run.shape)
+    m.row_ptr.copy_(torch.from_numpy(rp))
+    m.col_idx[: ci.size].copy_(torch.from_numpy(ci))
+    ws = torch.empty(fva.fva_tiles_workspace_bytes(run.shape), dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fva.fva_build_tiles(run.shape, m, ws, fva.FVA_ORDER_LPT, st)
+    o = torch.empty_like(run.layer.qh)
+    fva.fva_sparse_attn(run.shape, run.layer.qh, run.layer.kh, run.layer.vh, m, o, 0.0, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    perm, _ = O.hilbert_perm(wl.T, wl.Hg, wl.Wg)
+    qh, kh, vh = C.hilbert_bhnd(L, perm)
+    want = O.assemble(O.block_sparse_attention(qh, kh, vh, rp.astype(np.int64), ci.astype(np.int64)),
+                      wl.B, wl.H, wl.N, wl.d)
+    return o.float().cpu().numpy().astype(np.float64), want, vh
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_single_key_block_returns_its_value(d):
+    # N = 64*4 + 1: every row keeps only the 1-key tail block, so o = v[last] (bf16-rounded)
+    wl = synth.custom_workload(1, 1, 257, 2, d, "bf16", seed=38)
+    got, want, vh = _custom_mask_run(wl, lambda bh, a: [4])
+    _tol(wl, got, want, "one-key")
+    np.testing.assert_allclose(got[:, :, :, :], np.broadcast_to(vh[:, :, 256:257, :], got.shape), rtol=0, atol=1e-2)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_disjoint_pair_lists_and_all_blocks(d):
+    # rows 2t and 2t+1 keep disjoint lists (worst case for the pair union), plus all-block rows
+    wl = synth.custom_workload(3, 12, 12, 2, d, "bf16", seed=39)   # N = 432, nB = 7
+    got, want, _ = _custom_mask_run(wl, lambda bh, a: [a] if a % 2 == 0 else ([b for b in range(7) if b != a - 1]))
+    _tol(wl, got, want, "disjoint")
+    got, want, _ = _custom_mask_run(wl, lambda bh, a: list(range(7)))
+    _tol(wl, got, want, "all-blocks")
+
+
+@pytest.mark.parametrize("wid", [1, 3, 2])
+def test_sparse_full_size_sampled(wid):
+    """Full-size workloads in the benchmark's launch configuration; sampled query blocks."""
+    wl = synth.WORKLOADS[wid]
+    L = C.layer(wid)
+    run = C.GpuRun(wl, L)
+    g = run.mask_np()
+    got = run.layer
+    import torch
+    got.attend()
+    torch.cuda.synchronize()
+    assert run.status() == 0
+    BH, nB = wl.B * wl.H, wl.nB
+    rows = C.sample_rows(g["row_ptr"], BH, nB, 6, seed=wid)
+    perm, _ = O.hilbert_perm(wl.T, wl.Hg, wl.Wg)
+    max_err, sum_err, n = 0.0, 0.0, 0
+    heads = sorted({bh for bh, _ in rows})
+    for bh in heads:
+        qh = O.reorder(L.q[:, :, bh:bh + 1], perm)[0, 0]
+        kh = O.reorder(L.k[:, :, bh:bh + 1], perm)[0, 0]
+        vh = O.reorder(L.v[:, :, bh:bh + 1], perm)[0, 0]
+        for (b2, a) in rows:
+            if b2 != bh:
+                continue
+            keys = O.block_keys(O.row_list(g["row_ptr"], g["col_idx"], bh * nB + a), wl.N)
+            lo, hi = a * 64, min(a * 64 + 64, wl.N)
+            want = O.attention_rows(qh[lo:hi], kh, vh, keys, 1.0 / np.sqrt(wl.d))
+            gv = got.oh[0, bh, lo:hi].float().cpu().numpy().astype(np.float64)
+            diff = np.abs(gv - want)
+            max_err = max(max_err, float(diff.max()))
+            sum_err += float(diff.sum())
+            n += diff.size
+    mean_err = sum_err / n
+    print(f"{wl.name}: sampled {len(rows)} query blocks max-abs {max_err:.3e} mean-abs {mean_err:.3e}")
+    assert max_err <= C.BF16_MAX_ABS and mean_err <= C.BF16_MEAN_ABS
+
+
+def test_dense_full_size_sampled_480p():
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import fva
+    wl = synth.WORKLOADS[1]
+    L = C.layer(1)
+    run = C.GpuRun(wl, L)
+    o = torch.empty_like(run.layer.qh)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fva.fva_dense_attn(run.shape, run.layer.qh, run.layer.kh, run.layer.vh, o, 0.0, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    perm, _ = O.hilbert_perm(wl.T, wl.Hg, wl.Wg)
+    rng = np.random.default_rng(5)
+    for bh in rng.choice(wl.H, size=3, replace=False):
+        qh = O.reorder(L.q[:, :, bh:bh + 1], perm)[0, 0]
+        kh = O.reorder(L.k[:, :, bh:bh + 1], perm)[0, 0]
+        vh = O.reorder(L.v[:, :, bh:bh + 1], perm)[0, 0]
+        rows = np.concatenate([rng.choice(wl.N, size=64, replace=False), [wl.N - 1]])
+        want = O.attention_rows(qh[rows], kh, vh, np.arange(wl.N), 1.0 / np.sqrt(wl.d))
+        gv = o[0, bh, torch.as_tensor(rows, device="cuda")].float().cpu().numpy()
+        mx, mean = C.err_stats(gv, want)
+        assert mx <= C.BF16_MAX_ABS and mean <= C.BF16_MEAN_ABS, (mx, mean)

@@ -1,0 +1,149 @@
+"""GPU parity: Top-p / Top-k_floor routing, CSR mask, per-head kept counts, tile lists and
+work lists (C ABI vs oracle).
+
+Masks must be bit-exact except rows the oracle flags as ambiguous (a cumulative mass
+within 1e-6 of p, or logits at the cut closer than 1e-9 relative); those are counted and
+reported, never silently accepted.
+"""
+import numpy as np
+import pytest
+
+from adaptive_block_sparse_hilbert_b200 import synth
+import oracle as O
+from tests import _common as C
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_mask(wl, L, p, k_floor):
+    perm, _ = O.hilbert_perm(wl.T, wl.Hg, wl.Wg)
+    pq, pk = C.oracle_pooled(L, perm)
+    return O.route(pq, pk, wl.d, p, k_floor, with_ambiguity=True)
+
+
+def _check_route(wl, L, p, k_floor, order=2, need_pool=False, max_amb_frac=1e-3):
+    run = C.GpuRun(wl, L, p=p, k_floor=k_floor, order=order, need_pool=need_pool)
+    assert run.status() == 0
+    g = run.mask_np()
+    o = _oracle_mask(wl, L, p, k_floor)
+    BH, nB = wl.B * wl.H, wl.nB
+    mism, amb = C.compare_masks(g, o, BH * nB)
+    n_amb = int(amb.sum())
+    print(f"{wl.name} p={p} kf={k_floor}: rows={BH * nB} mismatches={mism.size} ambiguous={n_amb} "
+          f"density={g['row_ptr'][-1] / (BH * nB * nB):.4f}")
+    assert np.all(amb[mism]), f"non-ambiguous mismatching rows: {mism[~amb[mism]][:10]}"
+    assert n_amb <= max(2, max_amb_frac * BH * nB)
+    if mism.size == 0:
+        np.testing.assert_array_equal(g["row_ptr"], o["row_ptr"])
+        np.testing.assert_array_equal(g["head_kept"], o["head_kept"])
+    # CSR structure
+    rp, ci = g["row_ptr"], g["col_idx"]
+    assert rp[0] == 0 and np.all(np.diff(rp) >= 1)
+    for r in range(0, BH * nB, max(1, (BH * nB) // 2000)):
+        lst = ci[rp[r]:rp[r + 1]]
+        assert np.all(np.diff(lst) > 0) and lst[0] >= 0 and lst[-1] < nB
+    np.testing.assert_array_equal(g["head_kept"], [rp[(h + 1) * nB] - rp[h * nB] for h in range(BH)])
+    # tiles: union + membership bits, costs, work list
+    n_pairs = (nB + 1) // 2
+    tiles = C.expected_tiles(rp, ci, BH, nB)
+    costs = np.array([len(t) for t in tiles])
+    np.testing.assert_array_equal(g["tile_cost"], costs)
+    np.testing.assert_array_equal(g["tile_ptr"], np.concatenate([[0], np.cumsum(costs)]))
+    np.testing.assert_array_equal(g["tile_col"], np.concatenate([np.array(t, dtype=np.int64) for t in tiles]))
+    np.testing.assert_array_equal(g["worklist"], C.expected_worklist(costs, BH, n_pairs, order))
+    return run, g, o
+
+
+SMALL = [
+    synth.WORKLOADS[0],
+    synth.custom_workload(3, 10, 13, 3, 64, "bf16", seed=21),
+    synth.custom_workload(2, 9, 9, 2, 128, "bf16", seed=22, tau=("logU", 2.0, 6.0)),
+    synth.custom_workload(2, 5, 7, 2, 64, "f32", seed=23),
+    synth.custom_workload(4, 20, 20, 2, 64, "bf16", seed=24, tau=("logU", 0.2, 0.4)),
+]
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+@pytest.mark.parametrize("p,kf", [(0.9, 2), (0.5, 0), (0.95, 4), (1.0, 0), (0.3, 5), (0.9, 1000), (1e-9, 0)])
+@pytest.mark.parametrize("order", [0, 1, 2])
+def test_route_small(wl, p, kf, order):
+    L = synth.make_layer(wl)
+    _check_route(wl, L, p, kf, order)
+
+
+def test_route_internal_pooling_matches():
+    wl = synth.custom_workload(3, 10, 13, 3, 64, "bf16", seed=25)
+    L = synth.make_layer(wl)
+    a = C.GpuRun(wl, L).mask_np()
+    b = C.GpuRun(wl, L, need_pool=True).mask_np()
+    for key in a:
+        np.testing.assert_array_equal(a[key], b[key])
+
+
+def test_equal_logits_lowest_index_and_closed_form():
+    """Constant Q and K: every logit in a row ties; L = max(ceil(p nB), k_floor), lowest indices."""
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import fva, pipeline
+    T, Hg, Wg, H, d = 4, 16, 16, 2, 64
+    s = fva.make_shape(1, H, d, T, Hg, Wg, "bf16")
+    N, nB = T * Hg * Wg, 16
+    q = torch.full((1, N, H, d), 0.5, dtype=torch.bfloat16, device="cuda")
+    for p, kf, L in [(0.9, 2, 15), (0.5, 0, 8), (0.5, 11, 11), (1.0, 0, 16), (0.01, 0, 1)]:
+        lay = pipeline.SparseAttentionLayer(s, p, kf)
+        lay.reorder_inputs(q, q, q)
+        lay.route()
+        torch.cuda.synchronize()
+        rp = lay.mask.row_ptr.cpu().numpy()
+        ci = lay.mask.col_idx.cpu().numpy()
+        assert int(lay.dev_status.item()) == 0
+        for r in range(H * nB):
+            assert ci[rp[r]:rp[r + 1]].tolist() == list(range(L)), (p, kf, r)
+
+
+def test_build_tiles_from_csr_matches_route():
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import fva
+    wl = synth.custom_workload(3, 10, 13, 3, 64, "bf16", seed=26)
+    L = synth.make_layer(wl)
+    run = C.GpuRun(wl, L)
+    g = run.mask_np()
+    m2 = fva.Mask.allocate(run.shape)
+    m2.row_ptr.copy_(run.layer.mask.row_ptr)
+    m2.col_idx.copy_(run.layer.mask.col_idx)
+    ws = torch.empty(fva.fva_tiles_workspace_bytes(run.shape), dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fva.fva_build_tiles(run.shape, m2, ws, 2, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    n = int(g["tile_ptr"][-1])
+    np.testing.assert_array_equal(m2.tile_ptr.cpu().numpy(), g["tile_ptr"])
+    np.testing.assert_array_equal(m2.tile_col[:n].cpu().numpy(), g["tile_col"])
+    np.testing.assert_array_equal(m2.worklist.cpu().numpy(), g["worklist"])
+    np.testing.assert_array_equal(m2.head_kept.cpu().numpy(), g["head_kept"])
+
+
+@pytest.mark.parametrize("wid", [1, 3, 2])
+def test_route_full_size(wid):
+    wl = synth.WORKLOADS[wid]
+    _check_route(wl, C.layer(wid), wl.p, wl.k_floor, order=2)
+
+
+@pytest.mark.parametrize("p", [0.8, 0.95])
+def test_route_720p_p_sweep(p):
+    wl = synth.WORKLOADS[2]
+    _check_route(wl, C.layer(2), p, wl.k_floor, order=2)
+
+
+def test_hetero_heads_density_split():
+    """Head-heterogeneity workload: the 20% flat heads (tau = 0.3) are far denser than the
+    concentrated ones; their share of kept blocks is reported (0.40 with this generator)."""
+    wl = synth.WORKLOADS[3]
+    L = C.layer(3)
+    run = C.GpuRun(wl, L)
+    hk = run.mask_np()["head_kept"]
+    flat = L.tau < 1.0
+    assert flat.sum() == round(0.2 * wl.H)
+    share = hk[flat].sum() / hk.sum()
+    print(f"flat-head share of kept blocks: {share:.3f}")
+    assert hk[flat].min() > 2 * hk[~flat].max()
+    assert share > 0.3
