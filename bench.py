@@ -205,7 +205,7 @@ def run_reference(args):
     vals = []
     sample = ""
     for i in range(args.warmup + args.steps):
-        ms, sample, _ = oracle_sample(wl, L, n_heads=1, rows_per_head=8, seed=i)
+        ms, sample, _ = oracle_sample(wl, L, n_heads=args.cpu_heads, rows_per_head=args.cpu_rows, seed=i)
         if i >= args.warmup:
             vals.append(ms)
     cores, threads = cpu_cores()
@@ -452,8 +452,8 @@ def main():
     ap.add_argument("--impl", default="fva", choices=["fva", "reference"])
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-heads", type=int, default=2)
-    ap.add_argument("--cpu-rows", type=int, default=24)
+    ap.add_argument("--cpu-heads", type=int, default=8)
+    ap.add_argument("--cpu-rows", type=int, default=4)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
