@@ -76,7 +76,8 @@ constexpr size_t attn_smem_bytes() {
   return 1024 /*alignment slack*/ + AttnCfg<D>::kSmemData + sizeof(AttnBars<D>);
 }
 
-template <int D, bool DENSE>
+// VF16: V and P in fp16 for P.V (else both bf16); Q and K are bf16 either way.
+template <int D, bool DENSE, bool VF16>
 __global__ void __launch_bounds__(kAttnThreads, 2)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                      const __grid_constant__ CUtensorMap tmv, __nv_bfloat16* __restrict__ out,
@@ -191,8 +192,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   } else if (warp == 5) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);
+      constexpr uint32_t idesc_qk = idesc_f16kind_f32(kBM, kBN, 0, 0, kFmtBF16);
+      constexpr uint32_t idesc_pv = idesc_f16kind_f32(kBM, D, 0, 1, VF16 ? kFmtF16 : kFmtBF16);
       bool ok = mbar_wait(&bar.q_full, 0, abort_flag, kWaitLimitNs);
       bool issued = false;
       auto issue_pv = [&](int i) -> bool {
@@ -310,13 +311,16 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           l_sum *= ex2_approx(m_ref - m_new);
           m_ref = m_new;
         }
+        // the row sum adds the rounded weights that P.V actually uses, so the
+        // normalised weights sum to one exactly
         float ls = 0.0f;
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const float p0 = ex2_approx(x[2 * c] - m_ref);
           const float p1 = ex2_approx(x[2 * c + 1] - m_ref);
-          ls += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
+          pk[c] = VF16 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+          const float2 r = VF16 ? unpack_f16x2(pk[c]) : unpack_bf16x2(pk[c]);
+          ls += r.x + r.y;
         }
         l_sum += ls;
       } else {
@@ -385,48 +389,57 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 3-D map over a [B*H, N, d] bf16 tensor, box = 64 elements (128 B) x 64 rows x 1.
-static bool make_map(CUtensorMap* map, const void* base, int64_t BH, int64_t N, int64_t d) {
+// 3-D map over a [B*H, N, d] 16-bit tensor, box = 64 elements (128 B) x 64 rows x 1.
+static bool make_map(CUtensorMap* map, const void* base, int64_t BH, int64_t N, int64_t d, bool f16) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(N * d * 2)};
   const cuuint32_t box[3] = {64, 64, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  const CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool DENSE>
+template <int D, bool DENSE, bool VF16>
 static cudaError_t launch_attn_t(const Dims& Dm, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                  const fva_mask* m, void* o, float scale_log2, int32_t* dev_status, cudaStream_t st) {
   const size_t smem = attn_smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<D, DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<D, DENSE, VF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(Dm.tiles);
-  attn_bf16_kernel<D, DENSE><<<grid, kAttnThreads, smem, st>>>(
+  attn_bf16_kernel<D, DENSE, VF16><<<grid, kAttnThreads, smem, st>>>(
       mq, mk, mv, static_cast<__nv_bfloat16*>(o), DENSE ? nullptr : m->tile_ptr, DENSE ? nullptr : m->tile_col,
       DENSE ? nullptr : m->worklist, static_cast<int>(Dm.N), static_cast<int>(Dm.nB), static_cast<int>(Dm.nPairs),
       scale_log2, dev_status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_bf16(const Dims& Dm, const void* q, const void* k, const void* v, const fva_mask* m,
-                             bool dense, void* o, float scale, int32_t* dev_status, cudaStream_t st) {
+template <int D>
+static cudaError_t launch_attn_d(const Dims& Dm, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                 bool v_f16, const fva_mask* m, bool dense, void* o, float scale_log2,
+                                 int32_t* dev_status, cudaStream_t st) {
+  if (v_f16) {
+    return dense ? launch_attn_t<D, true, true>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st)
+                 : launch_attn_t<D, false, true>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st);
+  }
+  return dense ? launch_attn_t<D, true, false>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st)
+               : launch_attn_t<D, false, false>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st);
+}
+
+cudaError_t launch_attn_bf16(const Dims& Dm, const void* q, const void* k, const void* v, bool v_f16,
+                             const fva_mask* m, bool dense, void* o, float scale, int32_t* dev_status,
+                             cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, Dm.BH, Dm.N, Dm.d) || !make_map(&mk, k, Dm.BH, Dm.N, Dm.d) ||
-      !make_map(&mv, v, Dm.BH, Dm.N, Dm.d))
+  if (!make_map(&mq, q, Dm.BH, Dm.N, Dm.d, false) || !make_map(&mk, k, Dm.BH, Dm.N, Dm.d, false) ||
+      !make_map(&mv, v, Dm.BH, Dm.N, Dm.d, v_f16))
     return cudaErrorInvalidValue;
   const float scale_log2 = scale * 1.4426950408889634f;
-  if (Dm.d == 128) {
-    return dense ? launch_attn_t<128, true>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st)
-                 : launch_attn_t<128, false>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st);
-  }
-  return dense ? launch_attn_t<64, true>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st)
-               : launch_attn_t<64, false>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st);
+  if (Dm.d == 128) return launch_attn_d<128>(Dm, mq, mk, mv, v_f16, m, dense, o, scale_log2, dev_status, st);
+  return launch_attn_d<64>(Dm, mq, mk, mv, v_f16, m, dense, o, scale_log2, dev_status, st);
 }
 
 }  // namespace fva

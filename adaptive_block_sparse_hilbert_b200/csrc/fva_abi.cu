@@ -28,7 +28,7 @@ bool make_dims(const fva_shape* s, Dims* out) {
   D.esize = s->dtype == FVA_BF16 ? 2 : 4;
   if (D.N > 0x7fffffffLL || D.rows > 0x7fffffffLL) return false;
   const int64_t row_bytes = D.d * D.esize;
-  if (row_bytes % 16 != 0 || row_bytes > 1024) return false;
+  if (row_bytes != 64 && row_bytes != 128 && row_bytes != 256 && row_bytes != 512 && row_bytes != 1024) return false;
   if (s->Hg > 65536 || s->Wg > 65536) return false;
   if (D.BH > 65535 || D.nB > 65535 * 8) return false;
   *out = D;
@@ -136,8 +136,9 @@ int fva_reorder(const fva_shape* s, const void* x_in_dev, void* x_out_dev, doubl
                 const int32_t* perm_dev, int direction, fva_stream_t stream) {
   Dims D;
   if (!s || !x_in_dev || !x_out_dev || !perm_dev) return FVA_ERR_INVALID_ARG;
-  if (direction != FVA_FWD && direction != FVA_INV) return FVA_ERR_INVALID_ARG;
-  if (direction == FVA_INV && pooled_dev) return FVA_ERR_INVALID_ARG;
+  if (direction != FVA_FWD && direction != FVA_INV && direction != FVA_FWD_F16) return FVA_ERR_INVALID_ARG;
+  if (direction != FVA_FWD && pooled_dev) return FVA_ERR_INVALID_ARG;
+  if (direction == FVA_FWD_F16 && s->dtype != FVA_BF16) return FVA_ERR_INVALID_ARG;
   if (!make_dims(s, &D)) return FVA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(x_in_dev) || !aligned16(x_out_dev) || (pooled_dev && !aligned16(pooled_dev)))
     return FVA_ERR_ALIGNMENT;
@@ -215,8 +216,8 @@ int fva_build_tiles(const fva_shape* s, const fva_mask* mask, int order, void* w
   return cuda_status(launch_build_tiles(D, mask, order, rs, dev_status, stream));
 }
 
-static int attn_common(const fva_shape* s, const void* q, const void* k, const void* v, const fva_mask* m, void* o,
-                       float scale, bool dense, int32_t* dev_status, fva_stream_t stream) {
+static int attn_common(const fva_shape* s, const void* q, const void* k, const void* v, int v_dtype,
+                       const fva_mask* m, void* o, float scale, bool dense, int32_t* dev_status, fva_stream_t stream) {
   Dims D;
   if (!s || !q || !k || !v || !o) return FVA_ERR_INVALID_ARG;
   if (!make_dims(s, &D)) return FVA_ERR_UNSUPPORTED_SHAPE;
@@ -224,10 +225,12 @@ static int attn_common(const fva_shape* s, const void* q, const void* k, const v
   if (o == q || o == k || o == v) return FVA_ERR_INVALID_ARG;
   if (!(scale > 0.0f)) scale = 1.0f / sqrtf(static_cast<float>(D.d));
   if (s->dtype == FVA_BF16) {
+    if (v_dtype != FVA_BF16 && v_dtype != FVA_F16) return FVA_ERR_INVALID_ARG;
     if (D.d != 64 && D.d != 128) return FVA_ERR_UNSUPPORTED_SHAPE;
     if (!dense && (!m || !m->tile_ptr || !m->tile_col || !m->worklist)) return FVA_ERR_INVALID_ARG;
-    return cuda_status(launch_attn_bf16(D, q, k, v, m, dense, o, scale, dev_status, stream));
+    return cuda_status(launch_attn_bf16(D, q, k, v, v_dtype == FVA_F16, m, dense, o, scale, dev_status, stream));
   }
+  if (v_dtype != FVA_F32) return FVA_ERR_INVALID_ARG;
   if (D.d != 32 && D.d != 64 && D.d != 128) return FVA_ERR_UNSUPPORTED_SHAPE;
   if (!dense && (!m || !m->row_ptr || !m->col_idx)) return FVA_ERR_INVALID_ARG;
   return cuda_status(launch_attn_f32(D, static_cast<const float*>(q), static_cast<const float*>(k),
@@ -235,14 +238,14 @@ static int attn_common(const fva_shape* s, const void* q, const void* k, const v
                                      dense ? nullptr : m->col_idx, dense, static_cast<float*>(o), scale, stream));
 }
 
-int fva_sparse_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev, const fva_mask* mask,
-                    void* o_dev, float scale, int32_t* dev_status, fva_stream_t stream) {
-  return attn_common(s, q_dev, k_dev, v_dev, mask, o_dev, scale, false, dev_status, stream);
+int fva_sparse_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev, int v_dtype,
+                    const fva_mask* mask, void* o_dev, float scale, int32_t* dev_status, fva_stream_t stream) {
+  return attn_common(s, q_dev, k_dev, v_dev, v_dtype, mask, o_dev, scale, false, dev_status, stream);
 }
 
-int fva_dense_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev, void* o_dev,
-                   float scale, int32_t* dev_status, fva_stream_t stream) {
-  return attn_common(s, q_dev, k_dev, v_dev, nullptr, o_dev, scale, true, dev_status, stream);
+int fva_dense_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev, int v_dtype,
+                   void* o_dev, float scale, int32_t* dev_status, fva_stream_t stream) {
+  return attn_common(s, q_dev, k_dev, v_dev, v_dtype, nullptr, o_dev, scale, true, dev_status, stream);
 }
 
 }  // extern "C"

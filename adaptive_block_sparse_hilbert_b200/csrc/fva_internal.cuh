@@ -45,7 +45,7 @@ cudaError_t launch_route(const Dims& D, const double* pq, const double* pk, doub
 cudaError_t launch_build_tiles(const Dims& D, const fva_mask* m, int order, const RouteScratch& ws,
                                int32_t* dev_status, cudaStream_t st);
 
-cudaError_t launch_attn_bf16(const Dims& D, const void* q, const void* k, const void* v,
+cudaError_t launch_attn_bf16(const Dims& D, const void* q, const void* k, const void* v, bool v_f16,
                              const fva_mask* m, bool dense, void* o, float scale,
                              int32_t* dev_status, cudaStream_t st);
 cudaError_t launch_attn_f32(const Dims& D, const float* q, const float* k, const float* v,
@@ -181,14 +181,17 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return desc;
 }
 
-// Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulator.
-// c_format bits 4-5 = 1 (F32); a_format 7-9 = 1 (BF16); b_format 10-12 = 1 (BF16);
-// a_major bit 15, b_major bit 16 (1 = MN-major); N>>3 in bits 17-22; M>>4 in 24-28.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major, int b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn_major) << 15) |
+// Instruction descriptor, kind::f16 with an fp32 accumulator: c_format bits 4-5 = 1
+// (F32); a_format 7-9 and b_format 10-12 = ab_format (0 = F16, 1 = BF16; A and B always
+// share it); a_major bit 15, b_major bit 16 (1 = MN-major); N>>3 in bits 17-22; M>>4 in
+// bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_f16kind_f32(int M, int N, int a_mn_major, int b_mn_major,
+                                                         uint32_t ab_format) {
+  return (1u << 4) | (ab_format << 7) | (ab_format << 10) | (static_cast<uint32_t>(a_mn_major) << 15) |
          (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
+constexpr uint32_t kFmtF16 = 0, kFmtBF16 = 1;
 
 #define FVA_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), \
                   "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
@@ -232,11 +235,28 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// bf16x2 pack: `lo` goes to the low 16 bits (element k), `hi` to the high (element k+1).
+// bf16x2 / f16x2 packs: `lo` goes to the low 16 bits (element k), `hi` to the high
+// (element k+1).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t v;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(v) : "f"(hi), "f"(lo));
   return v;
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t v;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(v) : "f"(hi), "f"(lo));
+  return v;
+}
+// The two floats a packed pair holds again (exact widening).
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t v) {
+  return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
+  float lo, hi;
+  asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(v));
+  return make_float2(lo, hi);
 }
 
 // Warp reductions with a fixed butterfly order (deterministic).

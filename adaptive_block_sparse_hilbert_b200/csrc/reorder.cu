@@ -128,113 +128,129 @@ __device__ __forceinline__ void add_vec<float>(double* acc, const uint4& v) {
 
 constexpr int kReorderThreads = 256;
 
+// Eight bf16 values -> eight fp16 values (exact in range, saturated to +-65504 outside).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = fminf(fmaxf(__uint_as_float(w[i] << 16), -65504.0f), 65504.0f);
+    const float hi = fminf(fmaxf(__uint_as_float(w[i] & 0xFFFF0000u), -65504.0f), 65504.0f);
+    o[i] = pack_f16x2(lo, hi);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // MODE 0: forward permute [B,N,H,d] -> [B,H,N,d] (+ pool)
 // MODE 1: inverse permute [B,H,N,d] -> [B,N,H,d]
 // MODE 2: pool only, input already [B,H,N,d]
-// One CTA per (block a, head h, batch b). VPR = 16-byte vectors per (token, head) row.
-template <typename T, int MODE, bool POOL>
+// MODE 3: forward permute with the output converted bf16 -> fp16
+// One CTA per (block a, head h, batch b); VPR = 16-byte vectors per (token, head) row.
+// Every thread keeps one vector column and loads all of its rows before storing any,
+// so a CTA has its whole 64-row block in flight.
+template <typename T, int MODE, bool POOL, int VPR>
 __global__ void __launch_bounds__(kReorderThreads) reorder_kernel(
     const uint8_t* __restrict__ x_in, uint8_t* __restrict__ x_out, double* __restrict__ pooled,
-    const int32_t* __restrict__ perm, int N, int H, int vpr) {
-  constexpr int EPV = 16 / sizeof(T);  // elements per 16-byte vector
-  extern __shared__ double red[];      // [rows_per_pass][vpr * EPV] when POOL
+    const int32_t* __restrict__ perm, int N, int H) {
+  constexpr int EPV = 16 / sizeof(T);          // elements per 16-byte vector
+  constexpr int RPP = kReorderThreads / VPR;   // rows per pass
+  constexpr int NPASS = (kBlock + RPP - 1) / RPP;
+  constexpr int64_t kRowBytes = VPR * 16;
+  constexpr int kWidth = VPR * EPV;            // = d
+  __shared__ double red[POOL ? RPP * kWidth : 1];
   const int a = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int64_t row_bytes = static_cast<int64_t>(vpr) * 16;
-  const int v = threadIdx.x % vpr;
-  const int r0 = threadIdx.x / vpr;
-  const int rpp = kReorderThreads / vpr;  // rows per pass
-  const bool active = r0 < rpp;           // threads beyond rpp*vpr idle
+  const int v = threadIdx.x % VPR;
+  const int r0 = threadIdx.x / VPR;
   const int row_lo = a * kBlock;
   const int n_valid = min(kBlock, N - row_lo);
-  double acc[EPV];
+  uint4 buf[NPASS];
 #pragma unroll
-  for (int i = 0; i < EPV; ++i) acc[i] = 0.0;
-
-  if (active) {
-    constexpr int kMaxPass = 16;  // rpp >= 4 (vpr <= 64), so 64/rpp <= 16
-    uint4 buf[kMaxPass];
-    const int n_pass = (kBlock + rpp - 1) / rpp;
-#pragma unroll
-    for (int ps = 0; ps < kMaxPass; ++ps) {
-      if (ps < n_pass) {
-        const int r = r0 + ps * rpp;
-        if (r < n_valid) {
-          const int i = row_lo + r;
-          const uint8_t* src;
-          if (MODE == 0) {
-            src = x_in + ((static_cast<int64_t>(b) * N + perm[i]) * H + h) * row_bytes;
-          } else {
-            src = x_in + ((static_cast<int64_t>(b) * H + h) * N + i) * row_bytes;
-          }
-          buf[ps] = __ldg(reinterpret_cast<const uint4*>(src) + v);
-        }
+  for (int ps = 0; ps < NPASS; ++ps) {
+    const int r = r0 + ps * RPP;
+    if (r < n_valid) {
+      const int i = row_lo + r;
+      const uint8_t* src;
+      if (MODE == 0 || MODE == 3) {
+        src = x_in + ((static_cast<int64_t>(b) * N + perm[i]) * H + h) * kRowBytes;
+      } else {
+        src = x_in + ((static_cast<int64_t>(b) * H + h) * N + i) * kRowBytes;
       }
+      buf[ps] = __ldg(reinterpret_cast<const uint4*>(src) + v);
     }
+  }
+  double acc[POOL ? EPV : 1];
+  if (POOL) {
 #pragma unroll
-    for (int ps = 0; ps < kMaxPass; ++ps) {
-      if (ps < n_pass) {
-        const int r = r0 + ps * rpp;
-        if (r < n_valid) {
-          const int i = row_lo + r;
-          if (MODE != 2) {
-            uint8_t* dst;
-            if (MODE == 0) {
-              dst = x_out + ((static_cast<int64_t>(b) * H + h) * N + i) * row_bytes;
-            } else {
-              dst = x_out + ((static_cast<int64_t>(b) * N + perm[i]) * H + h) * row_bytes;
-            }
-            reinterpret_cast<uint4*>(dst)[v] = buf[ps];
-          }
-          if (POOL) add_vec<T>(acc, buf[ps]);
+    for (int e = 0; e < EPV; ++e) acc[e] = 0.0;
+  }
+#pragma unroll
+  for (int ps = 0; ps < NPASS; ++ps) {
+    const int r = r0 + ps * RPP;
+    if (r < n_valid) {
+      const int i = row_lo + r;
+      if (MODE != 2) {
+        uint8_t* dst;
+        if (MODE == 0 || MODE == 3) {
+          dst = x_out + ((static_cast<int64_t>(b) * H + h) * N + i) * kRowBytes;
+        } else {
+          dst = x_out + ((static_cast<int64_t>(b) * N + perm[i]) * H + h) * kRowBytes;
         }
+        reinterpret_cast<uint4*>(dst)[v] = (MODE == 3) ? bf16x8_to_f16x8(buf[ps]) : buf[ps];
       }
+      if (POOL) add_vec<T>(acc, buf[ps]);
     }
   }
   if (POOL) {
-    const int width = vpr * EPV;  // = d
-    if (active) {
 #pragma unroll
-      for (int e = 0; e < EPV; ++e) red[r0 * width + v * EPV + e] = acc[e];
-    }
+    for (int e = 0; e < EPV; ++e) red[r0 * kWidth + v * EPV + e] = acc[e];
     __syncthreads();
-    // column sums over the rpp partial rows, fixed order
-    for (int c = threadIdx.x; c < width; c += kReorderThreads) {
+    // column sums over the RPP partial rows, fixed order
+    for (int c = threadIdx.x; c < kWidth; c += kReorderThreads) {
       double s = 0.0;
-      for (int r = 0; r < rpp; ++r) s += red[r * width + c];
-      pooled[((static_cast<int64_t>(b) * H + h) * gridDim.x + a) * width + c] = s / static_cast<double>(n_valid);
+#pragma unroll 8
+      for (int r = 0; r < RPP; ++r) s += red[r * kWidth + c];
+      pooled[((static_cast<int64_t>(b) * H + h) * gridDim.x + a) * kWidth + c] = s / static_cast<double>(n_valid);
     }
   }
+}
+
+template <typename T, int VPR>
+static cudaError_t launch_reorder_v(const Dims& D, const void* x_in, void* x_out, double* pooled,
+                                    const int32_t* perm, int mode, cudaStream_t st) {
+  const dim3 grid(static_cast<unsigned>(D.nB), static_cast<unsigned>(D.H), static_cast<unsigned>(D.B));
+  const uint8_t* in = static_cast<const uint8_t*>(x_in);
+  uint8_t* out = static_cast<uint8_t*>(x_out);
+  const int N = static_cast<int>(D.N), H = static_cast<int>(D.H);
+  if (mode == 0 && pooled) {
+    reorder_kernel<T, 0, true, VPR><<<grid, kReorderThreads, 0, st>>>(in, out, pooled, perm, N, H);
+  } else if (mode == 0) {
+    reorder_kernel<T, 0, false, VPR><<<grid, kReorderThreads, 0, st>>>(in, out, nullptr, perm, N, H);
+  } else if (mode == 1) {
+    reorder_kernel<T, 1, false, VPR><<<grid, kReorderThreads, 0, st>>>(in, out, nullptr, perm, N, H);
+  } else if (mode == 3) {
+    reorder_kernel<T, 3, false, VPR><<<grid, kReorderThreads, 0, st>>>(in, out, nullptr, perm, N, H);
+  } else {
+    reorder_kernel<T, 2, true, VPR><<<grid, kReorderThreads, 0, st>>>(in, nullptr, pooled, nullptr, N, H);
+  }
+  return cudaGetLastError();
 }
 
 template <typename T>
 static cudaError_t launch_reorder_t(const Dims& D, const void* x_in, void* x_out, double* pooled,
                                     const int32_t* perm, int mode, cudaStream_t st) {
-  const int vpr = static_cast<int>(D.d * sizeof(T) / 16);
-  const int rpp = kReorderThreads / vpr;
-  const dim3 grid(static_cast<unsigned>(D.nB), static_cast<unsigned>(D.H), static_cast<unsigned>(D.B));
-  const size_t smem = pooled ? static_cast<size_t>(rpp) * D.d * sizeof(double) : 0;
-  const uint8_t* in = static_cast<const uint8_t*>(x_in);
-  uint8_t* out = static_cast<uint8_t*>(x_out);
-  const int N = static_cast<int>(D.N), H = static_cast<int>(D.H);
-  if (mode == 0 && pooled) {
-    cudaFuncSetAttribute(reorder_kernel<T, 0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(smem));
-    reorder_kernel<T, 0, true><<<grid, kReorderThreads, smem, st>>>(in, out, pooled, perm, N, H, vpr);
-  } else if (mode == 0) {
-    reorder_kernel<T, 0, false><<<grid, kReorderThreads, 0, st>>>(in, out, nullptr, perm, N, H, vpr);
-  } else if (mode == 1) {
-    reorder_kernel<T, 1, false><<<grid, kReorderThreads, 0, st>>>(in, out, nullptr, perm, N, H, vpr);
-  } else {
-    cudaFuncSetAttribute(reorder_kernel<T, 2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(smem));
-    reorder_kernel<T, 2, true><<<grid, kReorderThreads, smem, st>>>(in, nullptr, pooled, nullptr, N, H, vpr);
+  switch (D.d * static_cast<int64_t>(sizeof(T)) / 16) {
+    case 4: return launch_reorder_v<T, 4>(D, x_in, x_out, pooled, perm, mode, st);
+    case 8: return launch_reorder_v<T, 8>(D, x_in, x_out, pooled, perm, mode, st);
+    case 16: return launch_reorder_v<T, 16>(D, x_in, x_out, pooled, perm, mode, st);
+    case 32: return launch_reorder_v<T, 32>(D, x_in, x_out, pooled, perm, mode, st);
+    case 64: return launch_reorder_v<T, 64>(D, x_in, x_out, pooled, perm, mode, st);
+    default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_reorder(const Dims& D, const void* x_in, void* x_out, double* pooled,
                            const int32_t* perm, int direction, cudaStream_t st) {
-  const int mode = direction == FVA_FWD ? 0 : 1;
+  const int mode = direction == FVA_FWD ? 0 : (direction == FVA_INV ? 1 : 3);
   if (D.esize == 2) return launch_reorder_t<__nv_bfloat16>(D, x_in, x_out, pooled, perm, mode, st);
   return launch_reorder_t<float>(D, x_in, x_out, pooled, perm, mode, st);
 }

@@ -32,8 +32,10 @@ FVA_DEVERR_BAD_LIST = 3
 
 FVA_F32 = 0
 FVA_BF16 = 1
+FVA_F16 = 2
 FVA_FWD = 0
 FVA_INV = 1
+FVA_FWD_F16 = 2
 FVA_ORDER_NATURAL = 0
 FVA_ORDER_LPT = 1
 FVA_ORDER_HEAD_LPT = 2
@@ -82,8 +84,8 @@ def _load():
         "fva_pool": (i32, [S, P, P, P]),
         "fva_route": (i32, [S, P, P, P, P, dbl, i32, i32, M, P, sz, P, P]),
         "fva_build_tiles": (i32, [S, M, i32, P, sz, P, P]),
-        "fva_sparse_attn": (i32, [S, P, P, P, M, P, flt, P, P]),
-        "fva_dense_attn": (i32, [S, P, P, P, P, flt, P, P]),
+        "fva_sparse_attn": (i32, [S, P, P, P, i32, M, P, flt, P, P]),
+        "fva_dense_attn": (i32, [S, P, P, P, i32, P, flt, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -212,15 +214,21 @@ def fva_build_tiles(s, mask: Mask, workspace, order=FVA_ORDER_HEAD_LPT, dev_stat
                                                    ws_bytes, _ptr(dev_status), _stream(stream)))
 
 
-def fva_sparse_attn(s, q, k, v, mask: Mask, o, scale=0.0, dev_status=None, stream=None):
+def _dtype_code(t):
+    return {torch.float32: FVA_F32, torch.bfloat16: FVA_BF16, torch.float16: FVA_F16}[t.dtype]
+
+
+def fva_sparse_attn(s, q, k, v, mask: Mask, o, scale=0.0, dev_status=None, stream=None, v_dtype=None):
     m = mask.c() if isinstance(mask, Mask) else mask
-    _check("fva_sparse_attn", _lib.fva_sparse_attn(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(m),
+    vd = _dtype_code(v) if v_dtype is None else int(v_dtype)
+    _check("fva_sparse_attn", _lib.fva_sparse_attn(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), vd, ctypes.byref(m),
                                                    _ptr(o), float(scale), _ptr(dev_status), _stream(stream)))
 
 
-def fva_dense_attn(s, q, k, v, o, scale=0.0, dev_status=None, stream=None):
-    _check("fva_dense_attn", _lib.fva_dense_attn(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(o), float(scale),
-                                                 _ptr(dev_status), _stream(stream)))
+def fva_dense_attn(s, q, k, v, o, scale=0.0, dev_status=None, stream=None, v_dtype=None):
+    vd = _dtype_code(v) if v_dtype is None else int(v_dtype)
+    _check("fva_dense_attn", _lib.fva_dense_attn(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), vd, _ptr(o),
+                                                 float(scale), _ptr(dev_status), _stream(stream)))
 
 
 def call_raw(name, *args):

@@ -14,7 +14,7 @@ from . import fva
 
 class SparseAttentionLayer:
     def __init__(self, shape: fva.fva_shape, p: float, k_floor: int, order: int = fva.FVA_ORDER_HEAD_LPT,
-                 device: str = "cuda"):
+                 device: str = "cuda", v_fp16: bool = True):
         self.shape = shape
         self.p = float(p)
         self.k_floor = int(k_floor)
@@ -29,7 +29,10 @@ class SparseAttentionLayer:
         self.inv = torch.empty(self.N, dtype=torch.int32, device=device)
         self.qh = torch.empty(bhnd, dtype=dt, device=device)
         self.kh = torch.empty(bhnd, dtype=dt, device=device)
-        self.vh = torch.empty(bhnd, dtype=dt, device=device)
+        # bf16 layers keep the Hilbert-ordered V in fp16 so P.V runs with fp16 P (8x finer
+        # rounding of the attention weights than bf16); the conversion is fused into the reorder
+        self.v_fp16 = bool(v_fp16) and s.dtype == fva.FVA_BF16
+        self.vh = torch.empty(bhnd, dtype=torch.float16 if self.v_fp16 else dt, device=device)
         self.oh = torch.empty(bhnd, dtype=dt, device=device)
         self.pooled_q = torch.empty((s.B, s.H, self.nB, s.d), dtype=torch.float64, device=device)
         self.pooled_k = torch.empty_like(self.pooled_q)
@@ -43,7 +46,7 @@ class SparseAttentionLayer:
         s = self.shape
         fva.fva_reorder(s, q, self.qh, self.pooled_q, self.perm, fva.FVA_FWD, stream)
         fva.fva_reorder(s, k, self.kh, self.pooled_k, self.perm, fva.FVA_FWD, stream)
-        fva.fva_reorder(s, v, self.vh, None, self.perm, fva.FVA_FWD, stream)
+        fva.fva_reorder(s, v, self.vh, None, self.perm, fva.FVA_FWD_F16 if self.v_fp16 else fva.FVA_FWD, stream)
 
     def route(self, stream=None):
         fva.fva_route(self.shape, None, None, self.pooled_q, self.pooled_k, self.p, self.k_floor, self.mask,

@@ -66,8 +66,11 @@ enum {
   FVA_DEVERR_BAD_LIST = 3   /* a tile list entry was out of range */
 };
 
-enum { FVA_F32 = 0, FVA_BF16 = 1 };
-enum { FVA_FWD = 0, FVA_INV = 1 };
+/* Element types. FVA_F16 appears only as the type of a Hilbert-ordered V (see
+ * FVA_FWD_F16 and the v_dtype argument of the attention entry points). */
+enum { FVA_F32 = 0, FVA_BF16 = 1, FVA_F16 = 2 };
+/* Reorder directions: forward, inverse, forward with the output converted bf16 -> fp16. */
+enum { FVA_FWD = 0, FVA_INV = 1, FVA_FWD_F16 = 2 };
 /* Order of the attention work list (tiles are launched in this order). */
 enum {
   FVA_ORDER_NATURAL = 0,    /* tile id order */
@@ -138,7 +141,10 @@ FVA_API int fva_hilbert_perm(const fva_shape* s, int32_t* perm_dev, int32_t* inv
  *            [64a, min(64a+64, N)) in float64 (exact sum of the inputs, then / n_a).
  *   FVA_INV: x_out[b, perm[i], h, :] = x_in[b, h, i, :]   ([B,H,N,d] -> [B,N,H,d]);
  *            pooled_dev must be NULL.
- * Element type from s->dtype; d * sizeof(elem) must be a multiple of 16 and <= 1024.
+ *   FVA_FWD_F16: as FVA_FWD for a bf16 input, with x_out written as float16 (exact for
+ *            |x| < 65504, saturated to +-65504 beyond); pooled_dev must be NULL. This is
+ *            how V is prepared for the fp16 P.V path of the attention kernel.
+ * Element type from s->dtype; d * sizeof(elem) must be 64, 128, 256, 512 or 1024 bytes.
  * x_in and x_out must not overlap.
  */
 FVA_API int fva_reorder(const fva_shape* s, const void* x_in_dev, void* x_out_dev, double* pooled_dev,
@@ -186,18 +192,23 @@ FVA_API int fva_build_tiles(const fva_shape* s, const fva_mask* mask, int order,
  * Block-sparse attention ([aixai] sparse-attention section: only the kept key blocks of
  * a query block are computed). For each query i in block a of (b, h):
  *   o_i = sum_j softmax_j(scale * q_i . k_j) v_j  over the valid keys j of the kept blocks
- * (no causal mask). q, k, v, o: [B,H,N,d] Hilbert order, dtype s->dtype (bf16: d in
- * {64, 128}, fp32 accumulation, bf16 output; fp32: d % 4 == 0, d <= 128).
+ * (no causal mask). q, k, o: [B,H,N,d] Hilbert order, dtype s->dtype; v: [B,H,N,d] of
+ * type v_dtype.
+ *   s->dtype == FVA_BF16 (tensor cores, d in {64, 128}, fp32 accumulation, bf16 output):
+ *     v_dtype == FVA_F16: P is rounded to fp16 for P.V (the accurate path; prepare V
+ *                         with fva_reorder(FVA_FWD_F16));
+ *     v_dtype == FVA_BF16: P is rounded to bf16 for P.V.
+ *   s->dtype == FVA_F32 (CUDA cores, d in {32, 64, 128}): v_dtype must be FVA_F32.
  * scale <= 0 selects 1/sqrt(d). Reads mask->tile_ptr, tile_col, worklist (bf16) or
  * mask->row_ptr, col_idx (fp32). o must not overlap q, k or v.
  */
 FVA_API int fva_sparse_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev,
-                    const fva_mask* mask, void* o_dev, float scale, int32_t* dev_status,
-                    fva_stream_t stream);
+                            int v_dtype, const fva_mask* mask, void* o_dev, float scale, int32_t* dev_status,
+                            fva_stream_t stream);
 
 /* Dense attention (every block kept): the in-house density-1 reference. Same layouts. */
 FVA_API int fva_dense_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev,
-                   void* o_dev, float scale, int32_t* dev_status, fva_stream_t stream);
+                           int v_dtype, void* o_dev, float scale, int32_t* dev_status, fva_stream_t stream);
 
 #ifdef __cplusplus
 }

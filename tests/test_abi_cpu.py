@@ -99,7 +99,16 @@ def test_host_validation_before_any_launch():
                         None, None) == fva.FVA_ERR_WORKSPACE
     # bf16 attention supports d in {64, 128} only
     s96 = fva.make_shape(1, 2, 96, 4, 16, 16, "bf16")
-    assert fva.call_raw("fva_dense_attn", ctypes.byref(s96), one, one, one, P(4096), ctypes.c_float(0.0), None,
-                        None) == fva.FVA_ERR_UNSUPPORTED_SHAPE
-    assert fva.call_raw("fva_sparse_attn", ctypes.byref(s), one, one, one, None, P(4096), ctypes.c_float(0.0), None,
-                        None) == fva.FVA_ERR_INVALID_ARG
+    assert fva.call_raw("fva_dense_attn", ctypes.byref(s96), one, one, one, fva.FVA_F16, P(4096), ctypes.c_float(0.0),
+                        None, None) == fva.FVA_ERR_UNSUPPORTED_SHAPE
+    assert fva.call_raw("fva_sparse_attn", ctypes.byref(s), one, one, one, fva.FVA_F32, None, P(4096),
+                        ctypes.c_float(0.0), None, None) == fva.FVA_ERR_INVALID_ARG
+    # v_dtype must match: fp32 layers take fp32 V; bf16 layers take bf16 or fp16 V
+    assert fva.call_raw("fva_dense_attn", ctypes.byref(s), one, one, one, fva.FVA_F16, P(4096), ctypes.c_float(0.0),
+                        None, None) == fva.FVA_ERR_INVALID_ARG
+    sb = fva.make_shape(1, 2, 64, 4, 16, 16, "bf16")
+    assert fva.call_raw("fva_dense_attn", ctypes.byref(sb), one, one, one, fva.FVA_F32, P(4096), ctypes.c_float(0.0),
+                        None, None) == fva.FVA_ERR_INVALID_ARG
+    # fp16 conversion is a forward reorder of bf16 data only
+    assert fva.call_raw("fva_reorder", ctypes.byref(s), one, P(48), None, one, fva.FVA_FWD_F16, None) == \
+        fva.FVA_ERR_INVALID_ARG

@@ -65,6 +65,28 @@ def test_sparse_and_dense_small(wl):
     _tol(wl, _run_dense(run), O.dense_attention(qh, kh, vh), "dense")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_bf16_v_path(d):
+    """The kernel variant that rounds P to bf16 (V kept in bf16) also meets the tolerance."""
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import fva
+    wl = synth.custom_workload(3, 10, 13, 2, d, "bf16", seed=40)
+    L = synth.make_layer(wl)
+    run = C.GpuRun(wl, L)
+    vb = torch.empty(run.layer.vh.shape, dtype=torch.bfloat16, device="cuda")
+    fva.fva_reorder(run.shape, run.v, vb, None, run.layer.perm, fva.FVA_FWD)
+    o = torch.empty_like(run.layer.qh)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fva.fva_sparse_attn(run.shape, run.layer.qh, run.layer.kh, vb, run.layer.mask, o, 0.0, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    g = run.mask_np()
+    perm, _ = O.hilbert_perm(wl.T, wl.Hg, wl.Wg)
+    qh, kh, vh = C.hilbert_bhnd(L, perm)
+    want = O.assemble(O.block_sparse_attention(qh, kh, vh, g["row_ptr"], g["col_idx"]), wl.B, wl.H, wl.N, wl.d)
+    _tol(wl, o.float().cpu().numpy().astype(np.float64), want, "sparse-bf16V")
+
+
 def test_end_to_end_raster_output():
     """forward(): reorder -> route -> attention -> inverse reorder equals the oracle in raster order."""
     import torch
