@@ -86,6 +86,7 @@ const char* fva_status_string(int status) {
     case FVA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     case FVA_ERR_WORKSPACE: return "workspace too small";
     case FVA_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case FVA_ERR_TOO_LARGE: return "shape needs more scratch than the fixed no-alloc array holds";
     default: return "unknown status";
   }
 }

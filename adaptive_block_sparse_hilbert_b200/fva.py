@@ -24,6 +24,8 @@ FVA_ERR_CUDA = -4
 FVA_ERR_DEVICE_TIMEOUT = -5
 FVA_ERR_WORKSPACE = -6
 FVA_ERR_ALIGNMENT = -7
+FVA_ERR_TOO_LARGE = -8
+ROUTE_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 FVA_DEVERR_NONE = 0
 FVA_DEVERR_TIMEOUT = 1
@@ -84,6 +86,7 @@ def _load():
         "fva_pool": (i32, [S, P, P, P]),
         "fva_route": (i32, [S, P, P, P, P, dbl, i32, i32, M, P, sz, P, P]),
         "fva_build_tiles": (i32, [S, M, i32, P, sz, P, P]),
+        "fva_route_noalloc": (i32, [S, P, P, P, P, dbl, i32, i32, M, P, P]),
         "fva_sparse_attn": (i32, [S, P, P, P, i32, M, P, flt, P, P]),
         "fva_dense_attn": (i32, [S, P, P, P, i32, P, flt, P, P]),
     }
@@ -98,7 +101,7 @@ _lib = _load()
 EXPORTED = (
     "fva_status_string", "fva_version", "fva_num_tokens", "fva_num_blocks", "fva_num_tiles", "fva_mask_capacity",
     "fva_tile_capacity", "fva_route_workspace_bytes", "fva_tiles_workspace_bytes", "fva_hilbert_perm", "fva_reorder",
-    "fva_pool", "fva_route", "fva_build_tiles", "fva_sparse_attn", "fva_dense_attn",
+    "fva_pool", "fva_route", "fva_build_tiles", "fva_sparse_attn", "fva_dense_attn", "fva_route_noalloc",
 )
 
 
@@ -205,6 +208,16 @@ def fva_route(s, q, k, pooled_q, pooled_k, p, k_floor, mask: Mask, workspace, or
     _check("fva_route", _lib.fva_route(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(pooled_q), _ptr(pooled_k), float(p),
                                        int(k_floor), int(order), ctypes.byref(m), _ptr(workspace), ws_bytes,
                                        _ptr(dev_status), _stream(stream)))
+
+
+def fva_route_noalloc(s, q, k, pooled_q, pooled_k, p, k_floor, mask: Mask, order=FVA_ORDER_HEAD_LPT,
+                      dev_status=None, stream=None):
+    """fva_route without a workspace, for callers that cannot allocate device memory: the
+    scratch is a fixed 64 MiB array inside libfva (see include/fva.h)."""
+    m = mask.c() if isinstance(mask, Mask) else mask
+    _check("fva_route_noalloc", _lib.fva_route_noalloc(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(pooled_q),
+                                                       _ptr(pooled_k), float(p), int(k_floor), int(order),
+                                                       ctypes.byref(m), _ptr(dev_status), _stream(stream)))
 
 
 def fva_build_tiles(s, mask: Mask, workspace, order=FVA_ORDER_HEAD_LPT, dev_status=None, stream=None):

@@ -55,7 +55,8 @@ enum {
   FVA_ERR_CUDA = -4,              /* a CUDA runtime/driver call failed */
   FVA_ERR_DEVICE_TIMEOUT = -5,    /* reported through dev_status only */
   FVA_ERR_WORKSPACE = -6,         /* workspace smaller than the query function says */
-  FVA_ERR_ALIGNMENT = -7          /* a device pointer is not 16-byte aligned */
+  FVA_ERR_ALIGNMENT = -7,         /* a device pointer is not 16-byte aligned */
+  FVA_ERR_TOO_LARGE = -8          /* the shape needs more scratch than fva_route_noalloc holds */
 };
 
 /* Codes written to dev_status by kernels. */
@@ -209,6 +210,32 @@ FVA_API int fva_sparse_attn(const fva_shape* s, const void* q_dev, const void* k
 /* Dense attention (every block kept): the in-house density-1 reference. Same layouts. */
 FVA_API int fva_dense_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev,
                            int v_dtype, void* o_dev, float scale, int32_t* dev_status, fva_stream_t stream);
+
+/*
+ * Routing without a caller-provided workspace. The pages have no counterpart of this
+ * entry point; it exists for callers that cannot allocate device memory: a plugin inside
+ * a host application whose allocator owns all device memory, a service that forbids
+ * allocation after start-up to keep its footprint fixed, or any caller that holds only
+ * its input and output buffers.
+ * Same arguments and results as fva_route minus the workspace: the scratch lives in one
+ * fixed device array inside the library, FVA_ROUTE_NOALLOC_SCRATCH_BYTES (64 MiB) on
+ * every GPU that loads the library, held until the process exits. Nothing is allocated
+ * (no cudaMalloc/cudaFree, no allocating library call).
+ *   - Shapes whose fva_route_workspace_bytes(s, pooled == NULL) exceeds the array return
+ *     FVA_ERR_TOO_LARGE before anything is enqueued (e.g. 48 heads x 275 blocks fit;
+ *     40 heads x 512 blocks do not).
+ *   - The first call on a device looks up the array's device address with that device
+ *     current (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call uses the same array and leaves its contents behind; every byte a call
+ *     reads is written earlier in the same call. Calls whose work overlaps on the GPU
+ *     (other streams, other host threads, the same device) race on the array: order them
+ *     on one stream or synchronise between them.
+ */
+#define FVA_ROUTE_NOALLOC_SCRATCH_BYTES (64ull << 20)
+FVA_API int fva_route_noalloc(const fva_shape* s, const void* q_bhnd_dev, const void* k_bhnd_dev,
+                              const double* pooled_q_dev, const double* pooled_k_dev, double p, int k_floor,
+                              int order, const fva_mask* mask, int32_t* dev_status, fva_stream_t stream);
 
 #ifdef __cplusplus
 }
