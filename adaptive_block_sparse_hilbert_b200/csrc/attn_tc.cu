@@ -37,6 +37,13 @@ constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 64;   // keys per step (one key block)
 constexpr uint32_t kTmemCols = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Every kPolyEvery-th pair of scores can take exp2 on the FMA pipe instead of MUFU (build
+// option; 0 = never). Measured on B200 at d = 128, moving 1/8 .. 1/2 of the exponentials
+// to the polynomial made the kernel slower: the softmax is issue/latency bound, not MUFU bound.
+#ifndef FVA_POLY_EVERY
+#define FVA_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = FVA_POLY_EVERY;
 
 // Bounded wait taken by a whole warp: the result is the same on every lane, so the
 // warp stays converged for the .sync.aligned TMEM instructions that follow.
@@ -273,19 +280,25 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       tc_fence_after();
       uint32_t pk[32];
       if (keep) {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(lane_base + sb * 64, r0);
-        tmem_ld32(lane_base + sb * 64 + 32, r1);
-        const int nvalid = (kb == nB - 1) ? (N - kb * kBN) : kBN;
-        float x[64];
+        uint32_t r[64];
+        tmem_ld64(lane_base + sb * 64, r);
+        if (kb == nB - 1) {  // ragged last key block: keys past N score -inf
+          const int nvalid = N - kb * kBN;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] = (c < nvalid) ? __uint_as_float(r0[c]) * scale_log2 : -INFINITY;
-          x[c + 32] = (c + 32 < nvalid) ? __uint_as_float(r1[c]) * scale_log2 : -INFINITY;
+          for (int c = 0; c < 64; ++c)
+            if (c >= nvalid) r[c] = 0xFF800000u;
         }
-        float mx = x[0];
+        // row maximum of the raw scores: three-input max in four independent chains
+        float mx4[4];
 #pragma unroll
-        for (int c = 1; c < 64; ++c) mx = fmaxf(mx, x[c]);
+        for (int q = 0; q < 4; ++q) mx4[q] = __uint_as_float(r[q]);
+#pragma unroll
+        for (int c = 4; c < 64; c += 8) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            mx4[q] = fmax3(mx4[q], __uint_as_float(r[c + 2 * q]), __uint_as_float(r[c + 2 * q + 1]));
+        }
+        const float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * scale_log2;
         const float m_new = fmaxf(m_ref, mx);
         const bool need = m_new > m_ref + 8.0f;
         const bool need_o = need && (l_sum > 0.0f);
@@ -311,18 +324,29 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           l_sum *= ex2_approx(m_ref - m_new);
           m_ref = m_new;
         }
-        // the row sum adds the rounded weights that P.V actually uses, so the
-        // normalised weights sum to one exactly
-        float ls = 0.0f;
+        // p = 2^(s * scale * log2 e - m_ref) on pairs of scores: one packed FFMA, then
+        // either two MUFU.EX2 or (every kPolyEvery-th pair) the FMA-pipe polynomial, which
+        // keeps the MUFU pipe from being the step's bottleneck; the row sum runs in two
+        // packed accumulators
+        const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
+        const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
+        uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float p0 = ex2_approx(x[2 * c] - m_ref);
-          const float p1 = ex2_approx(x[2 * c + 1] - m_ref);
-          pk[c] = VF16 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
-          const float2 r = VF16 ? unpack_f16x2(pk[c]) : unpack_bf16x2(pk[c]);
-          ls += r.x + r.y;
+          const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])),
+                                            sc2, nm2));
+          uint64_t p2;
+          if (kPolyEvery > 0 && (c % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+            p2 = exp2_poly_pair(x.x, x.y);
+          } else {
+            p2 = f2_pack(ex2_approx(x.x), ex2_approx(x.y));
+          }
+          const float2 p = f2_unpack(p2);
+          pk[c] = VF16 ? pack_f16x2(p.x, p.y) : pack_bf16x2(p.x, p.y);
+          acc2[c & 1] = f2_add(acc2[c & 1], p2);
         }
-        l_sum += ls;
+        const float2 la = f2_unpack(f2_add(acc2[0], acc2[1]));
+        l_sum += la.x + la.y;
       } else {
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;

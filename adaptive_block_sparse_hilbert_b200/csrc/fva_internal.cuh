@@ -209,6 +209,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr)
       : "memory");
 }
+// Load 64 consecutive 32-bit TMEM columns of this thread's lane and wait for them.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : FVA_R8(0), FVA_R8(8), FVA_R8(16), FVA_R8(24), FVA_R8(32), FVA_R8(40), FVA_R8(48), FVA_R8(56)
+      : "r"(taddr)
+      : "memory");
+}
 // Store 32 consecutive 32-bit TMEM columns of this thread's lane and wait for the store.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
@@ -257,6 +270,57 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
       : "=f"(lo), "=f"(hi)
       : "r"(v));
   return make_float2(lo, hi);
+}
+
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic) ------------------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return make_float2(lo, hi);
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of floats on the FMA pipe (no MUFU): x = j + f with j = rint(x) and
+// f in [-1/2, 1/2]; 2^f by a degree-4 polynomial (coefficients fitted for this library
+// by weighted least squares in relative error on Chebyshev nodes; max relative error
+// 2.7e-6 in fp32 Horner form), then j is added to the exponent field. Inputs below -126
+// are clamped to -126 (result ~1e-38); inputs are at most 2^8 here.
+__device__ __forceinline__ uint64_t exp2_poly_pair(float x0, float x1) {
+  const float magic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+  const uint64_t xc = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t t = f2_add(xc, f2_pack(magic, magic));
+  const uint64_t j = f2_add(t, f2_pack(-magic, -magic));
+  const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), xc);
+  uint64_t p = f2_fma(f2_pack(0.009570096619427204f, 0.009570096619427204f), f,
+                      f2_pack(0.05591785907745361f, 0.05591785907745361f));
+  p = f2_fma(p, f, f2_pack(0.240247443318367f, 0.240247443318367f));
+  p = f2_fma(p, f, f2_pack(0.6931217908859253f, 0.6931217908859253f));
+  p = f2_fma(p, f, f2_pack(0.9999992847442627f, 0.9999992847442627f));
+  // bits(t) = bits(1.5 * 2^23) + j, and bits(1.5 * 2^23) << 23 == 0 modulo 2^32
+  const float2 tf = f2_unpack(t);
+  const float2 pf = f2_unpack(p);
+  const uint32_t lo = __float_as_uint(pf.x) + (__float_as_uint(tf.x) << 23);
+  const uint32_t hi = __float_as_uint(pf.y) + (__float_as_uint(tf.y) << 23);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
 // Warp reductions with a fixed butterfly order (deterministic).

@@ -23,15 +23,17 @@ namespace fva {
 // ---------------------------------------------------------------------------------
 // Block logits
 // ---------------------------------------------------------------------------------
-constexpr int kST = 64;  // output tile (rows and columns)
-constexpr int kSK = 16;  // d-chunk staged per step
+constexpr int kST = 64;   // output tile (rows and columns)
+constexpr int kSK = 16;   // d-chunk staged per step
+constexpr int kSP = kST + 2;  // padded row: transposed stores hit distinct banks, rows stay 16-B aligned
 
+// grid: (ceil(nB/64), ceil(nB/64), B*H); 256 threads, each a 4x4 block of logits.
 __global__ void __launch_bounds__(256) route_scores_kernel(const double* __restrict__ pq,
                                                            const double* __restrict__ pk,
                                                            double* __restrict__ S, int nB, int d,
                                                            double sqrt_d) {
-  __shared__ __align__(16) double As[kSK][kST];
-  __shared__ __align__(16) double Bs[kSK][kST];
+  __shared__ __align__(16) double As[kSK][kSP];
+  __shared__ __align__(16) double Bs[kSK][kSP];
   const int bh = blockIdx.z;
   const int a0 = blockIdx.y * kST, b0 = blockIdx.x * kST;
   const double* Q = pq + static_cast<int64_t>(bh) * nB * d;
@@ -43,12 +45,21 @@ __global__ void __launch_bounds__(256) route_scores_kernel(const double* __restr
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
 
+  // each thread stages two consecutive d-elements of one row of each tile (d is even)
+  const int lr = threadIdx.x >> 3;        // 0..31: row within a half tile
+  const int lc = (threadIdx.x & 7) * 2;   // 0..14: d offset within the chunk
   for (int i0 = 0; i0 < d; i0 += kSK) {
-    for (int e = threadIdx.x; e < kST * kSK; e += 256) {
-      const int r = e / kSK, c = e % kSK;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int r = lr + 32 * half;
       const int ga = a0 + r, gb = b0 + r;
-      As[c][r] = (ga < nB && i0 + c < d) ? Q[static_cast<int64_t>(ga) * d + i0 + c] : 0.0;
-      Bs[c][r] = (gb < nB && i0 + c < d) ? K[static_cast<int64_t>(gb) * d + i0 + c] : 0.0;
+      double2 qa = make_double2(0.0, 0.0), kb = make_double2(0.0, 0.0);
+      if (ga < nB && i0 + lc < d) qa = *reinterpret_cast<const double2*>(Q + static_cast<int64_t>(ga) * d + i0 + lc);
+      if (gb < nB && i0 + lc < d) kb = *reinterpret_cast<const double2*>(K + static_cast<int64_t>(gb) * d + i0 + lc);
+      As[lc][r] = qa.x;
+      As[lc + 1][r] = qa.y;
+      Bs[lc][r] = kb.x;
+      Bs[lc + 1][r] = kb.y;
     }
     __syncthreads();
 #pragma unroll 4
@@ -86,6 +97,7 @@ constexpr int kMaxLevels = 12;
 constexpr double kFix = 4503599627370496.0;     // 2^52: fixed-point unit of importance
 
 struct WarpArena {
+  double* s;          // [nB] the row's logits
   double* e;          // [nB] exp(s - max)
   uint64_t* hw;       // [kNBK] bucket mass (fixed point)
   int32_t* list;      // [nB] candidate block indices
@@ -95,6 +107,7 @@ struct WarpArena {
 
 __host__ __device__ inline size_t warp_arena_bytes(int nB, int nWords) {
   size_t b = 0;
+  b += align_up(static_cast<size_t>(nB) * 8, 16);
   b += align_up(static_cast<size_t>(nB) * 8, 16);
   b += kNBK * 8;
   b += align_up(static_cast<size_t>(nB) * 4, 16);
@@ -106,6 +119,8 @@ __host__ __device__ inline size_t warp_arena_bytes(int nB, int nWords) {
 __device__ inline WarpArena make_arena(uint8_t* base, int nB, int nWords) {
   WarpArena A;
   size_t off = 0;
+  A.s = reinterpret_cast<double*>(base + off);
+  off += align_up(static_cast<size_t>(nB) * 8, 16);
   A.e = reinterpret_cast<double*>(base + off);
   off += align_up(static_cast<size_t>(nB) * 8, 16);
   A.hw = reinterpret_cast<uint64_t*>(base + off);
@@ -124,8 +139,9 @@ __device__ __forceinline__ bool precedes(double sj, int j, double si, int i) {
   return sj > si || (sj == si && j < i);
 }
 
-__device__ __forceinline__ uint64_t fixed_mass(double e, double Z) {
-  return static_cast<uint64_t>((e / Z) * kFix);
+// importance e/Z in units of 2^-52 (zscale = 2^52 / Z), truncated
+__device__ __forceinline__ uint64_t fixed_mass(double e, double zscale) {
+  return static_cast<uint64_t>(e * zscale);
 }
 
 struct Pivot {
@@ -138,8 +154,9 @@ struct Pivot {
 // Find the pivot of the routing order for one row.
 // by_mass: the first position whose cumulative fixed-point mass reaches `pth`
 // (= p * 2^52); otherwise the position `cnt_target` (1-based) by count.
-__device__ Pivot select_pivot(const double* __restrict__ srow, const WarpArena& A, int nB, double smax,
-                              double smin, double Z, bool by_mass, double pth, int cnt_target) {
+__device__ Pivot select_pivot(const WarpArena& A, int nB, double smax, double smin, double zscale, bool by_mass,
+                              double pth, int cnt_target) {
+  const double* srow = A.s;
   const int lane = threadIdx.x & 31;
   uint64_t above_w = 0;
   int above_c = 0;
@@ -161,7 +178,7 @@ __device__ Pivot select_pivot(const double* __restrict__ srow, const WarpArena& 
       bk = bk < 0 ? 0 : (bk >= kNBK ? kNBK - 1 : bk);
       atomicAdd(&A.hcnt[bk], 1);
       if (by_mass) atomicAdd(reinterpret_cast<unsigned long long*>(&A.hw[bk]),
-                             static_cast<unsigned long long>(fixed_mass(A.e[b], Z)));
+                             static_cast<unsigned long long>(fixed_mass(A.e[b], zscale)));
     }
     __syncwarp();
     // lane owns buckets 4*lane .. 4*lane+3
@@ -274,12 +291,12 @@ __device__ Pivot select_pivot(const double* __restrict__ srow, const WarpArena& 
         const double sj = srow[bj];
         if (precedes(sj, bj, si, bi)) {
           ++rank;
-          if (by_mass) cw += fixed_mass(A.e[bj], Z);
+          if (by_mass) cw += fixed_mass(A.e[bj], zscale);
         }
       }
       bool ok;
       if (by_mass) {
-        cw += fixed_mass(A.e[bi], Z);
+        cw += fixed_mass(A.e[bi], zscale);
         ok = static_cast<double>(above_w + cw) >= pth;
       } else {
         ok = (above_c + rank + 1 == cnt_target);
@@ -328,10 +345,12 @@ __global__ void route_select_kernel(const double* __restrict__ S, int nB, int nW
 
   if (a < nB) {
     const int64_t row = static_cast<int64_t>(bh) * nB + a;
-    const double* srow = S + row * nB;
+    const double* grow = S + row * nB;
+    double* srow = A.s;
     double smax = -INFINITY, smin = INFINITY;
     for (int b = lane; b < nB; b += 32) {
-      const double s = srow[b];
+      const double s = grow[b];
+      srow[b] = s;
       smax = fmax(smax, s);
       smin = fmin(smin, s);
     }
@@ -344,6 +363,7 @@ __global__ void route_select_kernel(const double* __restrict__ S, int nB, int nW
       z += e;
     }
     const double Z = warp_sum_d(z);
+    const double zscale = kFix / Z;
     __syncwarp();
 
     const int L_k = k_floor < nB ? k_floor : nB;
@@ -354,11 +374,11 @@ __global__ void route_select_kernel(const double* __restrict__ S, int nB, int nW
     pv.s = smin;
     pv.b = nB - 1;
     if (!all) {
-      pv = select_pivot(srow, A, nB, smax, smin, Z, true, p * kFix, 0);
+      pv = select_pivot(A, nB, smax, smin, zscale, true, p * kFix, 0);
       if (!pv.found) {
         all = true;
       } else if (pv.L < L_k) {
-        pv = select_pivot(srow, A, nB, smax, smin, Z, false, 0.0, L_k);
+        pv = select_pivot(A, nB, smax, smin, zscale, false, 0.0, L_k);
         if (!pv.found) all = true;
       }
     }
@@ -613,9 +633,10 @@ __global__ void __launch_bounds__(256) tile_cost_kernel(const uint32_t* __restri
 // ---------------------------------------------------------------------------------
 static int select_rows_per_cta(const Dims& D) {
   const size_t arena = warp_arena_bytes(static_cast<int>(D.nB), static_cast<int>(D.nWords));
+  constexpr size_t kBudget = 224 * 1024;  // dynamic shared memory per CTA (227 KB maximum)
   int r = 8;
-  while (r > 2 && arena * r > 200 * 1024) r -= 2;
-  return (arena * r > 200 * 1024) ? 0 : r;
+  while (r > 2 && arena * r > kBudget) r -= 2;
+  return (arena * r > kBudget) ? 0 : r;
 }
 
 static cudaError_t launch_order_and_emit(const Dims& D, const fva_mask* m, int order, const RouteScratch& ws,
