@@ -36,7 +36,7 @@ constexpr int kAttnThreads = 192;
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 64;   // keys per step (one key block)
 constexpr uint32_t kTmemCols = 256;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 // Every kPolyEvery-th pair of scores can take exp2 on the FMA pipe instead of MUFU (build
 // option; 0 = never). Measured on B200 at d = 128, moving 1/8 .. 1/2 of the exponentials
 // to the polynomial made the kernel slower: the softmax is issue/latency bound, not MUFU bound.
@@ -47,8 +47,8 @@ constexpr int kPolyEvery = FVA_POLY_EVERY;
 
 // Bounded wait taken by a whole warp: the result is the same on every lane, so the
 // warp stays converged for the .sync.aligned TMEM instructions that follow.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, abort, kWaitLimitNs);
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                      const __grid_constant__ CUtensorMap tmv, __nv_bfloat16* __restrict__ out,
                      const int32_t* __restrict__ tile_ptr, const int32_t* __restrict__ tile_col,
                      const int32_t* __restrict__ worklist, int N, int nB, int nPairs, float scale_log2,
-                     int32_t* dev_status) {
+                     uint64_t kWaitLimitNs, uint32_t diag_flags, int32_t* dev_status) {
   using Cfg = AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -151,11 +151,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       int k_uses[Cfg::kStages], v_uses[Cfg::kStages];
       for (int s = 0; s < Cfg::kStages; ++s) k_uses[s] = v_uses[s] = 0;
       bool ok = true;
-      mbar_arrive_expect_tx(&bar.q_full, Cfg::kQBytes);
-      for (int c = 0; c < Cfg::kChunks; ++c)
-        for (int hf = 0; hf < 2; ++hf)
-          tma_load_3d(sQ + c * (kBM * 128) + hf * (64 * 128), &tmq, &bar.q_full, c * 64, t * kBM + hf * 64, bh);
-      last_q = 1;
+      // FVA_DIAG_WITHHOLD_Q: the Q tile is never requested, so every wait behind it runs out
+      if (!(diag_flags & FVA_DIAG_WITHHOLD_Q)) {
+        mbar_arrive_expect_tx(&bar.q_full, Cfg::kQBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c)
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_3d(sQ + c * (kBM * 128) + hf * (64 * 128), &tmq, &bar.q_full, c * 64, t * kBM + hf * 64, bh);
+        last_q = 1;
+      }
       for (int j = 0; j < n_iter && ok; ++j) {
         const int kb = DENSE ? j : (tile_col[list_base + j] >> 2);
         if (kb < 0 || kb >= nB) {
@@ -273,7 +276,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       const int kb = entry >> 2;
       const bool keep = (entry >> half) & 1;
       const int sb = j & 1;
-      if (!warp_wait(&bar.s_full[sb], (j >> 1) & 1, abort_flag)) {
+      if (!warp_wait(&bar.s_full[sb], (j >> 1) & 1, abort_flag, kWaitLimitNs)) {
         ok = false;
         break;
       }
@@ -305,7 +308,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         if (__any_sync(0xffffffffu, need_o)) {
           // O holds rows rescaled to the old maximum: wait for the PV of step j-1, then
           // O_row *= 2^(m_ref - m_new) for the rows whose maximum moved.
-          if (!warp_wait(&bar.pv_done, (j - 1) & 1, abort_flag)) {
+          if (!warp_wait(&bar.pv_done, (j - 1) & 1, abort_flag, kWaitLimitNs)) {
             ok = false;
             break;
           }
@@ -356,7 +359,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       mbar_arrive(&bar.p_full[sb]);
     }
     // ------------------------------------------------------------------ epilogue
-    if (ok && !warp_wait(&bar.o_full, 0, abort_flag)) ok = false;
+    if (ok && !warp_wait(&bar.o_full, 0, abort_flag, kWaitLimitNs)) ok = false;
     if (!ok) {
       report(dev_status, FVA_DEVERR_TIMEOUT);
       *abort_flag = 1;
@@ -397,6 +400,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 // ---------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------
+static uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
+static uint32_t g_diag_flags = 0;
+uint64_t attn_wait_limit_ns() { return g_wait_limit_ns; }
+uint32_t attn_diag_flags() { return g_diag_flags; }
+void set_attn_diagnostics(uint64_t ns, uint32_t flags) {
+  g_wait_limit_ns = ns == 0 ? kDefaultWaitLimitNs : ns;
+  g_diag_flags = flags;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -438,7 +450,7 @@ static cudaError_t launch_attn_t(const Dims& Dm, const CUtensorMap& mq, const CU
   attn_bf16_kernel<D, DENSE, VF16><<<grid, kAttnThreads, smem, st>>>(
       mq, mk, mv, static_cast<__nv_bfloat16*>(o), DENSE ? nullptr : m->tile_ptr, DENSE ? nullptr : m->tile_col,
       DENSE ? nullptr : m->worklist, static_cast<int>(Dm.N), static_cast<int>(Dm.nB), static_cast<int>(Dm.nPairs),
-      scale_log2, dev_status);
+      scale_log2, attn_wait_limit_ns(), attn_diag_flags(), dev_status);
   return cudaGetLastError();
 }
 

@@ -93,6 +93,10 @@ const char* fva_status_string(int status) {
 
 int fva_version(void) { return 100; }
 
+void fva_set_diagnostics(uint64_t wait_limit_ns, int flags) {
+  set_attn_diagnostics(wait_limit_ns, static_cast<uint32_t>(flags));
+}
+
 int64_t fva_num_tokens(const fva_shape* s) {
   Dims D;
   return make_dims(s, &D) ? D.N : -1;

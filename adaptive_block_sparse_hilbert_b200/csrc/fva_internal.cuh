@@ -48,6 +48,9 @@ cudaError_t launch_build_tiles(const Dims& D, const fva_mask* m, int order, cons
 cudaError_t launch_attn_bf16(const Dims& D, const void* q, const void* k, const void* v, bool v_f16,
                              const fva_mask* m, bool dense, void* o, float scale,
                              int32_t* dev_status, cudaStream_t st);
+uint64_t attn_wait_limit_ns();
+uint32_t attn_diag_flags();
+void set_attn_diagnostics(uint64_t wait_limit_ns, uint32_t flags);
 cudaError_t launch_attn_f32(const Dims& D, const float* q, const float* k, const float* v,
                             const int32_t* row_ptr, const int32_t* col_idx, bool dense, float* o,
                             float scale, cudaStream_t st);
@@ -97,15 +100,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait: true once the phase with this parity has completed; false if `abort`
-// became nonzero or about `limit_ns` passed (the caller then reports and unwinds).
+// became nonzero or about `limit_ns` passed (the caller then reports and unwinds). Each
+// try_wait may suspend the thread for a hardware-chosen time, so the clock is read after
+// every attempt.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_test(bar, parity)) return true;
+    if (mbar_test(bar, parity)) return true;
     if (*abort) return false;
     if (global_timer_ns() - t0 > limit_ns) return false;
   }

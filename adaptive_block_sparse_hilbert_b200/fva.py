@@ -74,6 +74,7 @@ def _load():
     sig = {
         "fva_status_string": (ctypes.c_char_p, [i32]),
         "fva_version": (i32, []),
+        "fva_set_diagnostics": (None, [ctypes.c_uint64, i32]),
         "fva_num_tokens": (i64, [S]),
         "fva_num_blocks": (i64, [S]),
         "fva_num_tiles": (i64, [S]),
@@ -99,7 +100,7 @@ def _load():
 
 _lib = _load()
 EXPORTED = (
-    "fva_status_string", "fva_version", "fva_num_tokens", "fva_num_blocks", "fva_num_tiles", "fva_mask_capacity",
+    "fva_status_string", "fva_version", "fva_set_diagnostics", "fva_num_tokens", "fva_num_blocks", "fva_num_tiles", "fva_mask_capacity",
     "fva_tile_capacity", "fva_route_workspace_bytes", "fva_tiles_workspace_bytes", "fva_hilbert_perm", "fva_reorder",
     "fva_pool", "fva_route", "fva_build_tiles", "fva_sparse_attn", "fva_dense_attn", "fva_route_noalloc",
 )
@@ -107,6 +108,15 @@ EXPORTED = (
 
 def lib():
     return _lib
+
+
+FVA_DIAG_WITHHOLD_Q = 1
+
+
+def fva_set_diagnostics(wait_limit_ns: int = 0, flags: int = 0) -> None:
+    """Attention-kernel diagnostics: wait time limit (0 = 2 s default) and flags
+    (FVA_DIAG_WITHHOLD_Q: skip the Q load so the waits behind it run out)."""
+    _lib.fva_set_diagnostics(int(wait_limit_ns), int(flags))
 
 
 def status_string(status: int) -> str:

@@ -109,6 +109,22 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ----------------------------------------------------------------------------------- ranks
+
+def ranks_max(values, dist_mod, device):
+    """Element-wise maximum of per-rank timings over all ranks (every rank gets the result)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_ms_per_layer(ms_per_step_max: float, world: int, layers_per_rank_step: int = 1) -> float:
+    """Replicas: every rank processes its own layer(s) per step, so the whole job finishes
+    world * layers_per_rank_step layers in the slowest rank's step time."""
+    return ms_per_step_max / (world * layers_per_rank_step)
+
+
 # ----------------------------------------------------------------------------------- schedule model
 
 def list_schedule(costs: np.ndarray, order: np.ndarray, slots: int):
@@ -257,7 +273,10 @@ def run_gpu(args):
     wl = synth.WORKLOADS[args.workload]
     if args.p is not None:
         wl = synth.Workload(**{**wl.__dict__, "p": args.p})
-    L = synth.make_layer(wl)
+    # the drift workload is a sequence of denoising steps, each a fresh layer that is
+    # re-routed and recomputed; the timed loop cycles through them
+    layers_np = [synth.make_layer(wl, st) for st in range(wl.steps)]
+    L = layers_np[0]
     s = fva.make_shape(wl.B, wl.H, wl.d, wl.T, wl.Hg, wl.Wg, wl.dtype)
     dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
 
@@ -269,13 +288,18 @@ def run_gpu(args):
     hq, hk, hv = host(L.q, L.q_bits), host(L.k, L.k_bits), host(L.v, L.v_bits)
     ho = torch.empty_like(hq).pin_memory()
     q, k, v = hq.to(dev), hk.to(dev), hv.to(dev)
+    qkv_steps = [(q, k, v)] + [tuple(host(a, b).to(dev) for a, b in ((X.q, X.q_bits), (X.k, X.k_bits), (X.v, X.v_bits)))
+                               for X in layers_np[1:]]
     o = torch.empty_like(q)
     layer = pipeline.SparseAttentionLayer(s, wl.p, wl.k_floor, device=dev)
     stream = torch.cuda.current_stream()
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    step_idx = [0]
 
     def step(marks=None):
+        q, k, v = qkv_steps[step_idx[0] % len(qkv_steps)]
+        step_idx[0] += 1
         if marks is not None:
             marks[0].record(stream)
         layer.reorder_inputs(q, k, v)
@@ -313,29 +337,52 @@ def run_gpu(args):
     total_ms = start.elapsed_time(end)
     clk = clocks.stop()
     if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = ranks_max([total_ms], dist, dev)[0]
         dist.barrier()
-        total_ms = float(t.item())
     status = int(layer.dev_status.item())
 
     stage = np.array([[m[j].elapsed_time(m[j + 1]) for j in range(4)] for m in marks])
     t_reorder, t_route, t_attn, t_inv = [float(np.mean(stage[:, j])) for j in range(4)]
     ms_step = total_ms / args.steps
 
-    # mask statistics and algorithmic work
-    rp = layer.mask.row_ptr.cpu().numpy().astype(np.int64)
+    # mask statistics and algorithmic work (averaged over the drift steps, which the timed
+    # loop visits equally often)
     nB, N, d, BH = wl.nB, wl.N, wl.d, wl.B * wl.H
-    kept = int(rp[-1])
     sizes = np.minimum(64, N - 64 * np.arange(nB)).astype(np.int64)
-    ci = layer.mask.col_idx[:kept].cpu().numpy().astype(np.int64)
-    counts = np.diff(rp)
-    a_idx = np.repeat(np.arange(BH * nB) % nB, counts)
-    kept_flops = float(4 * d * np.sum(sizes[a_idx] * sizes[ci]))
-    costs = layer.mask.tile_cost.cpu().numpy().astype(np.int64)
-    issued_flops = float(4 * d * 128 * 64 * costs.sum())
+
+    def mask_stats():
+        rp = layer.mask.row_ptr.cpu().numpy().astype(np.int64)
+        kept = int(rp[-1])
+        ci = layer.mask.col_idx[:kept].cpu().numpy().astype(np.int64)
+        a_idx = np.repeat(np.arange(BH * nB) % nB, np.diff(rp))
+        kf = float(4 * d * np.sum(sizes[a_idx] * sizes[ci]))
+        costs = layer.mask.tile_cost.cpu().numpy().astype(np.int64)
+        return kept, kf, costs, layer.mask.head_kept.cpu().numpy().astype(np.float64)
+
+    per_step = []
+    for qq, kk, vv in qkv_steps:
+        if len(qkv_steps) > 1:
+            layer.reorder_inputs(qq, kk, vv)
+            layer.route()
+        per_step.append(mask_stats())
+    kept = int(np.mean([x[0] for x in per_step]))
+    kept_flops = float(np.mean([x[1] for x in per_step]))
+    costs = per_step[0][2]
+    issued_flops = float(np.mean([4 * d * 128 * 64 * x[2].sum() for x in per_step]))
     dense_flops = float(4 * d * BH * N * N)
     reorder_bytes = float(6 * wl.B * N * wl.H * d * (2 if wl.dtype == "bf16" else 4) + 2 * BH * nB * d * 8)
+    drift = None
+    if len(per_step) > 1:
+        kept_heads = [x[3] for x in per_step]
+        swings = [np.abs(b - a) / np.maximum(a, 1.0) for a, b in zip(kept_heads[:-1], kept_heads[1:])]
+        drift = {"steps": wl.steps, "alphas": list(wl.alphas),
+                 "density_per_step": [round(float(x.sum()) / (BH * nB * nB), 4) for x in kept_heads],
+                 "max_head_density_change": round(float(max(x.max() for x in swings)), 4),
+                 "mean_head_density_change": round(float(np.mean([x.mean() for x in swings])), 4),
+                 "note": "value = reorder + routing + attention + inverse reorder per denoising step, "
+                         "each step a fresh layer"}
+        layer.reorder_inputs(q, k, v)  # step 0 again for the dense and end-to-end runs below
+        layer.route()
 
     pk, how = peaks()
     peak_tf = float(pk.get("bf16_tflops_sustained", pk.get("bf16_tflops")))
@@ -380,9 +427,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / n_e2e
     if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+        e2e_ms = ranks_max([e2e_ms], dist, dev)[0]
 
     sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
     imb = imbalance(costs, BH, (nB + 1) // 2, 2 * sm_count)
@@ -397,7 +442,7 @@ def run_gpu(args):
     if rank == 0:
         line = {
             "metric": METRIC,
-            "value": round(ms_step / world, 4),
+            "value": round(whole_job_ms_per_layer(ms_step, world), 4),
             "unit": "ms/layer",
             "n_gpus": world,
             "steps": args.steps,
@@ -433,6 +478,8 @@ def run_gpu(args):
             "clocks": clk,
             "dev_status": status,
         }
+        if drift is not None:
+            line["drift"] = drift
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)

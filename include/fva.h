@@ -114,6 +114,16 @@ typedef struct fva_mask {
 FVA_API const char* fva_status_string(int status);
 FVA_API int fva_version(void);
 
+/* Diagnostics of the attention kernels (process-wide; for failure-detection tests).
+ * wait_limit_ns: time limit of every mbarrier wait (default 2 s; 0 restores it). A wait
+ *   that runs out sets FVA_DEVERR_TIMEOUT in dev_status, and its CTA drains its own loads
+ *   and MMAs, frees TMEM and exits; the device stays usable.
+ * flags: FVA_DIAG_WITHHOLD_Q makes each CTA skip its Q tile load, so the waits behind it
+ *   can never complete and run out after wait_limit_ns (a wait on a flag nothing sets).
+ * fva_set_diagnostics(0, 0) restores normal operation. */
+enum { FVA_DIAG_WITHHOLD_Q = 1 };
+FVA_API void fva_set_diagnostics(uint64_t wait_limit_ns, int flags);
+
 /* Derived sizes; -1 for an invalid shape. */
 FVA_API int64_t fva_num_tokens(const fva_shape* s);
 FVA_API int64_t fva_num_blocks(const fva_shape* s);
