@@ -159,31 +159,53 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             tma_load_3d(sQ + c * (kBM * 128) + hf * (64 * 128), &tmq, &bar.q_full, c * 64, t * kBM + hf * 64, bh);
         last_q = 1;
       }
-      for (int j = 0; j < n_iter && ok; ++j) {
-        const int kb = DENSE ? j : (tile_col[list_base + j] >> 2);
-        if (kb < 0 || kb >= nB) {
+      // K runs kStages blocks ahead of V: the MMA warp needs K(j+1) before V(j), and a K
+      // stage is free as soon as its QK product has run, long before the V stage of the
+      // same step (whose PV waits for the softmax)
+      auto key_block = [&](int j, int* kb) -> bool {
+        *kb = DENSE ? j : (tile_col[list_base + j] >> 2);
+        if (*kb < 0 || *kb >= nB) {
           report(dev_status, FVA_DEVERR_BAD_LIST);
           *abort_flag = 1;
-          break;
+          return false;
         }
+        return true;
+      };
+      auto load_k = [&](int j) -> bool {
+        int kb;
+        if (!key_block(j, &kb)) return false;
         const int s = j % Cfg::kStages;
         const uint32_t use = static_cast<uint32_t>(j / Cfg::kStages);
         if (j >= Cfg::kStages && !mbar_wait(&bar.k_empty[s], (use - 1) & 1, abort_flag, kWaitLimitNs)) {
           ok = false;
-          break;
+          return false;
         }
         mbar_arrive_expect_tx(&bar.k_full[s], Cfg::kKVBytes);
         for (int c = 0; c < Cfg::kChunks; ++c)
           tma_load_3d(sK + s * Cfg::kKVBytes + c * (kBN * 128), &tmk, &bar.k_full[s], c * 64, kb * kBN, bh);
         ++k_uses[s];
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        int kb;
+        if (!key_block(j, &kb)) return false;
+        const int s = j % Cfg::kStages;
+        const uint32_t use = static_cast<uint32_t>(j / Cfg::kStages);
         if (j >= Cfg::kStages && !mbar_wait(&bar.v_empty[s], (use - 1) & 1, abort_flag, kWaitLimitNs)) {
           ok = false;
-          break;
+          return false;
         }
         mbar_arrive_expect_tx(&bar.v_full[s], Cfg::kKVBytes);
         for (int c = 0; c < Cfg::kChunks; ++c)
           tma_load_3d(sV + s * Cfg::kKVBytes + c * (kBN * 128), &tmv, &bar.v_full[s], c * 64, kb * kBN, bh);
         ++v_uses[s];
+        return true;
+      };
+      bool go = true;
+      for (int j = 0; j < Cfg::kStages && j < n_iter && go; ++j) go = load_k(j);
+      for (int j = 0; j < n_iter && go; ++j) {
+        go = load_v(j);
+        if (go && j + Cfg::kStages < n_iter) go = load_k(j + Cfg::kStages);
       }
       if (!ok) {
         report(dev_status, FVA_DEVERR_TIMEOUT);
