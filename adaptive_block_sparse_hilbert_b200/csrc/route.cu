@@ -23,15 +23,18 @@ namespace fva {
 // ---------------------------------------------------------------------------------
 // Block logits
 // ---------------------------------------------------------------------------------
-constexpr int kST = 64;   // output tile (rows and columns)
-constexpr int kSK = 16;   // d-chunk staged per step
-constexpr int kSP = kST + 2;  // padded row: transposed stores hit distinct banks, rows stay 16-B aligned
+constexpr int kST = 128;  // output tile (rows and columns)
+constexpr int kSK = 8;    // d-chunk staged per step (d is a multiple of 8)
+constexpr int kSP = kST + 2;  // padded row: transposed stores spread over banks, rows stay 16-B aligned
 
-// grid: (ceil(nB/64), ceil(nB/64), B*H); 256 threads, each a 4x4 block of logits.
-__global__ void __launch_bounds__(256) route_scores_kernel(const double* __restrict__ pq,
-                                                           const double* __restrict__ pk,
-                                                           double* __restrict__ S, int nB, int d,
-                                                           double sqrt_d) {
+// grid: (ceil(nB/128), ceil(nB/128), B*H); 256 threads in a 16 x 16 grid, each an 8 x 8
+// block of logits: rows {4 ty + i, 64 + 4 ty + i} and columns {4 tx + j, 64 + 4 tx + j},
+// i, j < 4, so every shared-memory operand read is a 16-byte pair and a warp's B reads are
+// contiguous. 16 operand loads per 64 DFMA per chunk column.
+__global__ void __launch_bounds__(256, 1) route_scores_kernel(const double* __restrict__ pq,
+                                                              const double* __restrict__ pk,
+                                                              double* __restrict__ S, int nB, int d,
+                                                              double sqrt_d) {
   __shared__ __align__(16) double As[kSK][kSP];
   __shared__ __align__(16) double Bs[kSK][kSP];
   const int bh = blockIdx.z;
@@ -39,52 +42,71 @@ __global__ void __launch_bounds__(256) route_scores_kernel(const double* __restr
   const double* Q = pq + static_cast<int64_t>(bh) * nB * d;
   const double* K = pk + static_cast<int64_t>(bh) * nB * d;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  double acc[4][4];
+  double acc[8][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
 
-  // each thread stages two consecutive d-elements of one row of each tile (d is even)
-  const int lr = threadIdx.x >> 3;        // 0..31: row within a half tile
-  const int lc = (threadIdx.x & 7) * 2;   // 0..14: d offset within the chunk
+  // each thread stages four consecutive d-elements of one row of each tile
+  const int lr = threadIdx.x >> 1;        // 0..127: row within the tile
+  const int lc = (threadIdx.x & 1) * 4;   // 0 or 4: d offset within the chunk
+  const int ga = a0 + lr, gb = b0 + lr;
   for (int i0 = 0; i0 < d; i0 += kSK) {
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int r = lr + 32 * half;
-      const int ga = a0 + r, gb = b0 + r;
-      double2 qa = make_double2(0.0, 0.0), kb = make_double2(0.0, 0.0);
-      if (ga < nB && i0 + lc < d) qa = *reinterpret_cast<const double2*>(Q + static_cast<int64_t>(ga) * d + i0 + lc);
-      if (gb < nB && i0 + lc < d) kb = *reinterpret_cast<const double2*>(K + static_cast<int64_t>(gb) * d + i0 + lc);
-      As[lc][r] = qa.x;
-      As[lc + 1][r] = qa.y;
-      Bs[lc][r] = kb.x;
-      Bs[lc + 1][r] = kb.y;
+    double2 q0 = make_double2(0.0, 0.0), q1 = q0, k0 = q0, k1 = q0;
+    if (ga < nB) {
+      const double2* src = reinterpret_cast<const double2*>(Q + static_cast<int64_t>(ga) * d + i0 + lc);
+      q0 = src[0];
+      q1 = src[1];
     }
+    if (gb < nB) {
+      const double2* src = reinterpret_cast<const double2*>(K + static_cast<int64_t>(gb) * d + i0 + lc);
+      k0 = src[0];
+      k1 = src[1];
+    }
+    As[lc][lr] = q0.x;
+    As[lc + 1][lr] = q0.y;
+    As[lc + 2][lr] = q1.x;
+    As[lc + 3][lr] = q1.y;
+    Bs[lc][lr] = k0.x;
+    Bs[lc + 1][lr] = k0.y;
+    Bs[lc + 2][lr] = k1.x;
+    Bs[lc + 3][lr] = k1.y;
     __syncthreads();
-#pragma unroll 4
+#pragma unroll
     for (int c = 0; c < kSK; ++c) {
-      const double2 a01 = *reinterpret_cast<const double2*>(&As[c][ty * 4]);
-      const double2 a23 = *reinterpret_cast<const double2*>(&As[c][ty * 4 + 2]);
-      const double2 b01 = *reinterpret_cast<const double2*>(&Bs[c][tx * 4]);
-      const double2 b23 = *reinterpret_cast<const double2*>(&Bs[c][tx * 4 + 2]);
-      const double av[4] = {a01.x, a01.y, a23.x, a23.y};
-      const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
+      double av[8], bv[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int h = 0; h < 2; ++h) {
+        const double2 a01 = *reinterpret_cast<const double2*>(&As[c][h * 64 + ty * 4]);
+        const double2 a23 = *reinterpret_cast<const double2*>(&As[c][h * 64 + ty * 4 + 2]);
+        const double2 b01 = *reinterpret_cast<const double2*>(&Bs[c][h * 64 + tx * 4]);
+        const double2 b23 = *reinterpret_cast<const double2*>(&Bs[c][h * 64 + tx * 4 + 2]);
+        av[4 * h] = a01.x;
+        av[4 * h + 1] = a01.y;
+        av[4 * h + 2] = a23.x;
+        av[4 * h + 3] = a23.y;
+        bv[4 * h] = b01.x;
+        bv[4 * h + 1] = b01.y;
+        bv[4 * h + 2] = b23.x;
+        bv[4 * h + 3] = b23.y;
+      }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fma(av[i], bv[j], acc[i][j]);
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fma(av[i], bv[j], acc[i][j]);
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int a = a0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int a = a0 + (i >> 2) * 64 + ty * 4 + (i & 3);
     if (a >= nB) continue;
+    double* dst = S + (static_cast<int64_t>(bh) * nB + a) * nB;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int b = b0 + tx * 4 + j;
-      if (b < nB) S[(static_cast<int64_t>(bh) * nB + a) * nB + b] = acc[i][j] / sqrt_d;
+    for (int j = 0; j < 8; ++j) {
+      const int b = b0 + (j >> 2) * 64 + tx * 4 + (j & 3);
+      if (b < nB) dst[b] = acc[i][j] / sqrt_d;
     }
   }
 }
@@ -533,18 +555,10 @@ __global__ void __launch_bounds__(256) order_head_lpt_kernel(const int32_t* __re
 // ---------------------------------------------------------------------------------
 // Emission of col_idx and tile_col from the bitmasks
 // ---------------------------------------------------------------------------------
-__device__ __forceinline__ int warp_exclusive_scan_i(int v, int* total) {
-  const int lane = threadIdx.x & 31;
-  int inc = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += n;
-  }
-  *total = __shfl_sync(0xffffffffu, inc, 31);
-  return inc - v;
-}
-
+// One warp per tile (query blocks 2t and 2t+1 of one (b, h)). The warp walks the two
+// rows' bitmasks one 32-block word at a time; lane i owns block 32 k + i, and its output
+// slot is the number of set bits below it, so every store instruction writes one
+// contiguous run of entries.
 __global__ void __launch_bounds__(256) emit_kernel(const uint32_t* __restrict__ bits, int nB, int nWords,
                                                    int nPairs, int64_t tiles, const int32_t* __restrict__ row_ptr,
                                                    const int32_t* __restrict__ tile_ptr, int32_t* col_idx,
@@ -557,35 +571,31 @@ __global__ void __launch_bounds__(256) emit_kernel(const uint32_t* __restrict__ 
   const int64_t rA = bh * nB + 2 * t;
   const bool hasB = 2 * t + 1 < nB;
   const int64_t rB = rA + 1;
-  const int64_t baseA = row_ptr[rA];
-  const int64_t baseB = hasB ? row_ptr[rB] : 0;
-  const int64_t baseT = tile_ptr[tile];
-  int runA = 0, runB = 0, runT = 0;
+  int32_t* outA = col_idx + row_ptr[rA];
+  int32_t* outB = hasB ? col_idx + row_ptr[rB] : nullptr;
+  int32_t* outT = tile_col + tile_ptr[tile];
+  const uint32_t below = (1u << lane) - 1u;
   for (int k0 = 0; k0 < nWords; k0 += 32) {
-    const int k = k0 + lane;
-    const uint32_t wa = k < nWords ? bits[rA * nWords + k] : 0u;
-    const uint32_t wb = (hasB && k < nWords) ? bits[rB * nWords + k] : 0u;
-    const uint32_t wu = wa | wb;
-    int totA, totB, totU;
-    const int oa = warp_exclusive_scan_i(__popc(wa), &totA);
-    const int ob = warp_exclusive_scan_i(__popc(wb), &totB);
-    const int ou = warp_exclusive_scan_i(__popc(wu), &totU);
-    int ia = 0, ib = 0, iu = 0;
-    uint32_t m = wu;
-    while (m) {
-      const int bit = __ffs(m) - 1;
-      m &= m - 1;
-      const int blk = 32 * k + bit;
-      const uint32_t inA = (wa >> bit) & 1u, inB = (wb >> bit) & 1u;
+    // lane q holds word k0 + q of both rows
+    const uint32_t myA = k0 + lane < nWords ? bits[rA * nWords + k0 + lane] : 0u;
+    const uint32_t myB = (hasB && k0 + lane < nWords) ? bits[rB * nWords + k0 + lane] : 0u;
+    const int kn = nWords - k0 < 32 ? nWords - k0 : 32;
+    for (int q = 0; q < kn; ++q) {
+      const uint32_t wa = __shfl_sync(0xffffffffu, myA, q);
+      const uint32_t wb = __shfl_sync(0xffffffffu, myB, q);
+      const uint32_t wu = wa | wb;
+      const int blk = 32 * (k0 + q) + lane;
+      const uint32_t inA = (wa >> lane) & 1u, inB = (wb >> lane) & 1u;
       if (write_rows) {
-        if (inA) col_idx[baseA + runA + oa + ia++] = blk;
-        if (inB) col_idx[baseB + runB + ob + ib++] = blk;
+        if (inA) outA[__popc(wa & below)] = blk;
+        if (inB) outB[__popc(wb & below)] = blk;
+        outA += __popc(wa);
+        if (hasB) outB += __popc(wb);
       }
-      tile_col[baseT + runT + ou + iu++] = (blk << 2) | static_cast<int>(inA) | (static_cast<int>(inB) << 1);
+      if ((wu >> lane) & 1u)
+        outT[__popc(wu & below)] = (blk << 2) | static_cast<int>(inA) | (static_cast<int>(inB) << 1);
+      outT += __popc(wu);
     }
-    runA += totA;
-    runB += totB;
-    runT += totU;
   }
 }
 
