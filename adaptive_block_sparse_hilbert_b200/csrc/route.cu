@@ -52,8 +52,9 @@ __global__ void __launch_bounds__(256, 1) route_scores_kernel(const double* __re
   const int lr = threadIdx.x >> 1;        // 0..127: row within the tile
   const int lc = (threadIdx.x & 1) * 4;   // 0 or 4: d offset within the chunk
   const int ga = a0 + lr, gb = b0 + lr;
-  for (int i0 = 0; i0 < d; i0 += kSK) {
-    double2 q0 = make_double2(0.0, 0.0), q1 = q0, k0 = q0, k1 = q0;
+  // the next chunk is loaded into registers while the current one is multiplied
+  double2 q0 = make_double2(0.0, 0.0), q1 = q0, k0 = q0, k1 = q0;
+  auto fetch = [&](int i0) {
     if (ga < nB) {
       const double2* src = reinterpret_cast<const double2*>(Q + static_cast<int64_t>(ga) * d + i0 + lc);
       q0 = src[0];
@@ -64,6 +65,9 @@ __global__ void __launch_bounds__(256, 1) route_scores_kernel(const double* __re
       k0 = src[0];
       k1 = src[1];
     }
+  };
+  fetch(0);
+  for (int i0 = 0; i0 < d; i0 += kSK) {
     As[lc][lr] = q0.x;
     As[lc + 1][lr] = q0.y;
     As[lc + 2][lr] = q1.x;
@@ -73,6 +77,7 @@ __global__ void __launch_bounds__(256, 1) route_scores_kernel(const double* __re
     Bs[lc + 2][lr] = k1.x;
     Bs[lc + 3][lr] = k1.y;
     __syncthreads();
+    if (i0 + kSK < d) fetch(i0 + kSK);
 #pragma unroll
     for (int c = 0; c < kSK; ++c) {
       double av[8], bv[8];
