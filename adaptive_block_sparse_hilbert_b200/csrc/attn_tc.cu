@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                      const __grid_constant__ CUtensorMap tmv, __nv_bfloat16* __restrict__ out,
                      const int32_t* __restrict__ tile_ptr, const int32_t* __restrict__ tile_col,
                      const int32_t* __restrict__ worklist, int N, int nB, int nPairs, float scale_log2,
-                     uint64_t kWaitLimitNs, uint32_t diag_flags, int32_t* dev_status) {
+                     uint64_t kWaitLimitNs, uint32_t diag_flags, int32_t* dev_status, int64_t* cta_trace) {
   using Cfg = AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     n_iter = tile_ptr[tile + 1] - list_base;
   }
 
+  const uint64_t t_start = cta_trace != nullptr && threadIdx.x == 0 ? global_timer_ns() : 0;
   if (threadIdx.x == 128) {
     tma_prefetch_desc(&tmq);
     tma_prefetch_desc(&tmk);
@@ -417,6 +418,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  if (cta_trace != nullptr && threadIdx.x == 0) {
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    int64_t* rec = cta_trace + 4 * static_cast<int64_t>(blockIdx.x);
+    rec[0] = smid;
+    rec[1] = n_iter;
+    rec[2] = static_cast<int64_t>(t_start);
+    rec[3] = static_cast<int64_t>(global_timer_ns());
+  }
 }
 
 // ---------------------------------------------------------------------------------
@@ -424,6 +434,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 // ---------------------------------------------------------------------------------
 static uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 static uint32_t g_diag_flags = 0;
+static int64_t* g_cta_trace = nullptr;
+static int64_t g_cta_trace_capacity = 0;
+void set_attn_cta_trace(int64_t* trace, int64_t capacity_ctas) {
+  g_cta_trace = trace;
+  g_cta_trace_capacity = capacity_ctas;
+}
+bool attn_cta_trace_fits(int64_t ctas) { return g_cta_trace == nullptr || g_cta_trace_capacity >= ctas; }
 uint64_t attn_wait_limit_ns() { return g_wait_limit_ns; }
 uint32_t attn_diag_flags() { return g_diag_flags; }
 void set_attn_diagnostics(uint64_t ns, uint32_t flags) {
@@ -472,7 +489,7 @@ static cudaError_t launch_attn_t(const Dims& Dm, const CUtensorMap& mq, const CU
   attn_bf16_kernel<D, DENSE, VF16><<<grid, kAttnThreads, smem, st>>>(
       mq, mk, mv, static_cast<__nv_bfloat16*>(o), DENSE ? nullptr : m->tile_ptr, DENSE ? nullptr : m->tile_col,
       DENSE ? nullptr : m->worklist, static_cast<int>(Dm.N), static_cast<int>(Dm.nB), static_cast<int>(Dm.nPairs),
-      scale_log2, attn_wait_limit_ns(), attn_diag_flags(), dev_status);
+      scale_log2, attn_wait_limit_ns(), attn_diag_flags(), dev_status, g_cta_trace);
   return cudaGetLastError();
 }
 

@@ -97,6 +97,13 @@ void fva_set_diagnostics(uint64_t wait_limit_ns, int flags) {
   set_attn_diagnostics(wait_limit_ns, static_cast<uint32_t>(flags));
 }
 
+int fva_set_cta_trace(int64_t* trace_dev, int64_t capacity_ctas) {
+  if ((trace_dev == nullptr) != (capacity_ctas == 0) || capacity_ctas < 0) return FVA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(trace_dev) % 8 != 0) return FVA_ERR_ALIGNMENT;
+  set_attn_cta_trace(trace_dev, capacity_ctas);
+  return FVA_OK;
+}
+
 int64_t fva_num_tokens(const fva_shape* s) {
   Dims D;
   return make_dims(s, &D) ? D.N : -1;
@@ -233,6 +240,7 @@ static int attn_common(const fva_shape* s, const void* q, const void* k, const v
     if (v_dtype != FVA_BF16 && v_dtype != FVA_F16) return FVA_ERR_INVALID_ARG;
     if (D.d != 64 && D.d != 128) return FVA_ERR_UNSUPPORTED_SHAPE;
     if (!dense && (!m || !m->tile_ptr || !m->tile_col || !m->worklist)) return FVA_ERR_INVALID_ARG;
+    if (!attn_cta_trace_fits(D.tiles)) return FVA_ERR_CAPACITY;
     return cuda_status(launch_attn_bf16(D, q, k, v, v_dtype == FVA_F16, m, dense, o, scale, dev_status, stream));
   }
   if (v_dtype != FVA_F32) return FVA_ERR_INVALID_ARG;

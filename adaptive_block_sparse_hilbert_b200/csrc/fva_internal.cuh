@@ -51,6 +51,8 @@ cudaError_t launch_attn_bf16(const Dims& D, const void* q, const void* k, const 
 uint64_t attn_wait_limit_ns();
 uint32_t attn_diag_flags();
 void set_attn_diagnostics(uint64_t wait_limit_ns, uint32_t flags);
+void set_attn_cta_trace(int64_t* trace, int64_t capacity_ctas);
+bool attn_cta_trace_fits(int64_t ctas);
 cudaError_t launch_attn_f32(const Dims& D, const float* q, const float* k, const float* v,
                             const int32_t* row_ptr, const int32_t* col_idx, bool dense, float* o,
                             float scale, cudaStream_t st);

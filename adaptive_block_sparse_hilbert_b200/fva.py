@@ -57,6 +57,11 @@ class fva_mask(ctypes.Structure):
                 ("tile_capacity", ctypes.c_int64), ("tile_cost", ctypes.c_void_p), ("worklist", ctypes.c_void_p)]
 
 
+class fva_rlb_move(ctypes.Structure):
+    _fields_ = [("head", ctypes.c_int32), ("from_rank", ctypes.c_int32), ("to_rank", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("gain_ms", ctypes.c_double)]
+
+
 class FvaError(RuntimeError):
     def __init__(self, fn: str, status: int):
         super().__init__(f"{fn} failed: {status_string(status)} ({status})")
@@ -75,6 +80,10 @@ def _load():
         "fva_status_string": (ctypes.c_char_p, [i32]),
         "fva_version": (i32, []),
         "fva_set_diagnostics": (None, [ctypes.c_uint64, i32]),
+        "fva_set_cta_trace": (i32, [P, i64]),
+        "fva_rlb_plan": (i32, [ctypes.POINTER(ctypes.c_double), i32, i32, dbl, dbl, dbl, i32,
+                               ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(fva_rlb_move), i32,
+                               ctypes.POINTER(ctypes.c_int)]),
         "fva_num_tokens": (i64, [S]),
         "fva_num_blocks": (i64, [S]),
         "fva_num_tiles": (i64, [S]),
@@ -103,6 +112,7 @@ EXPORTED = (
     "fva_status_string", "fva_version", "fva_set_diagnostics", "fva_num_tokens", "fva_num_blocks", "fva_num_tiles", "fva_mask_capacity",
     "fva_tile_capacity", "fva_route_workspace_bytes", "fva_tiles_workspace_bytes", "fva_hilbert_perm", "fva_reorder",
     "fva_pool", "fva_route", "fva_build_tiles", "fva_sparse_attn", "fva_dense_attn", "fva_route_noalloc",
+    "fva_set_cta_trace", "fva_rlb_plan",
 )
 
 
@@ -117,6 +127,38 @@ def fva_set_diagnostics(wait_limit_ns: int = 0, flags: int = 0) -> None:
     """Attention-kernel diagnostics: wait time limit (0 = 2 s default) and flags
     (FVA_DIAG_WITHHOLD_Q: skip the Q load so the waits behind it run out)."""
     _lib.fva_set_diagnostics(int(wait_limit_ns), int(flags))
+
+
+def fva_set_cta_trace(trace=None) -> None:
+    """Per-CTA trace of the bf16 attention kernels: `trace` is an int64 device tensor of
+    shape [ctas, 4] (SM id, list length, start ns, end ns per CTA), or None to stop."""
+    if trace is None:
+        st = _lib.fva_set_cta_trace(None, 0)
+    else:
+        if trace.dtype != torch.int64 or trace.dim() != 2 or trace.shape[1] != 4 or not trace.is_contiguous():
+            raise ValueError("trace must be a contiguous int64 tensor of shape [ctas, 4]")
+        st = _lib.fva_set_cta_trace(_ptr(trace), int(trace.shape[0]))
+    if st != 0:
+        raise FvaError("fva_set_cta_trace", st)
+
+
+def fva_rlb_plan(head_load_ms, n_ranks: int, comm_ms: float, sched_ms: float, threshold: float = 1.10,
+                 max_per_rank: int = 1):
+    """Runtime Load Balancing plan (host): returns (rank_of int32[n_heads], moves) with
+    moves = [(head, from_rank, to_rank, gain_ms)] in the order they are applied."""
+    import numpy as np
+    load = np.ascontiguousarray(head_load_ms, dtype=np.float64)
+    H = int(load.shape[0])
+    cap = max(1, min(H, n_ranks * max_per_rank))
+    rank_of = np.zeros(H, dtype=np.int32)
+    moves = (fva_rlb_move * cap)()
+    n = ctypes.c_int(0)
+    st = _lib.fva_rlb_plan(load.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), H, int(n_ranks), float(comm_ms),
+                           float(sched_ms), float(threshold), int(max_per_rank),
+                           rank_of.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), moves, cap, ctypes.byref(n))
+    if st != 0:
+        raise FvaError("fva_rlb_plan", st)
+    return rank_of, [(m.head, m.from_rank, m.to_rank, m.gain_ms) for m in moves[:n.value]]
 
 
 def status_string(status: int) -> str:

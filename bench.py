@@ -139,6 +139,54 @@ def list_schedule(costs: np.ndarray, order: np.ndarray, slots: int):
     return load
 
 
+def measured_sm_imbalance(trace: np.ndarray, sm_count: int):
+    """SM-level balance of one traced attention launch. trace: int64 [ctas, 4] rows of
+    (SM id, list length in key blocks, start ns, end ns). Work per SM is the sum of the
+    list lengths of the CTAs it ran; finish per SM is its last CTA's end, measured from the
+    launch's first start. SMs that ran nothing count as zero work and zero finish."""
+    sm = trace[:, 0].astype(np.int64)
+    work = np.bincount(sm, weights=trace[:, 1].astype(np.float64), minlength=sm_count)[:sm_count]
+    t0 = int(trace[:, 2].min())
+    finish = np.zeros(sm_count)
+    np.maximum.at(finish, sm, (trace[:, 3] - t0).astype(np.float64))
+    span = float(trace[:, 3].max() - t0)
+    return {"sm_work_max_over_mean": round(float(work.max() / work.mean()), 4),
+            "sm_work_max_over_min": round(float(work.max() / max(work.min(), 1.0)), 4),
+            "sm_finish_mean_over_span": round(float(finish.mean() / span), 4) if span > 0 else None,
+            "span_ms": round(span / 1e6, 3), "ctas": int(trace.shape[0]), "sms": int(sm_count)}
+
+
+PEER_COPY_GBS = 770.0  # measured NVLink peer copy, GB/s per direction (B200, this pool)
+
+
+def rlb_report(costs: np.ndarray, BH: int, n_pairs: int, t_attn_ms: float, head_bytes: float, ranks: int = 8):
+    """Runtime Load Balancing on a virtual `ranks`-way head split of this layer: per-head
+    load = its tiles' list lengths x the measured time per tile step on one GPU; P = the
+    head's Q, K, V in and O out at the peer-copy rate; C = the planner's host time."""
+    import time
+    from adaptive_block_sparse_hilbert_b200 import fva
+    steps = costs.reshape(BH, n_pairs).sum(axis=1).astype(np.float64)
+    unit = t_attn_ms / max(float(steps.sum()), 1.0)
+    load = steps * unit
+    comm = head_bytes / (PEER_COPY_GBS * 1e9) * 1e3
+    t0 = time.perf_counter()
+    rank_of, moves = fva.fva_rlb_plan(load, ranks, comm, 0.0)
+    sched = (time.perf_counter() - t0) * 1e3
+    rank_of, moves = fva.fva_rlb_plan(load, ranks, comm, sched)  # with C measured
+
+    def stats(r):
+        Lr = np.bincount(r, weights=load, minlength=ranks)
+        return {"max_over_mean": round(float(Lr.max() / Lr.mean()), 4),
+                "max_over_min": round(float(Lr.max() / Lr.min()), 4) if Lr.min() > 0 else None,
+                "makespan_ms": round(float(Lr.max()), 3)}
+
+    home = (np.arange(BH) * ranks) // BH
+    return {"ranks": ranks, "heads": BH, "before": stats(home), "after": stats(rank_of.astype(np.int64)),
+            "moves": [[int(h), int(a), int(b)] for h, a, b, _ in moves],
+            "comm_ms_per_head": round(comm, 4), "sched_ms": round(sched, 4),
+            "note": "virtual split on one GPU; ranks run their heads at this GPU's measured rate"}
+
+
 def imbalance(costs: np.ndarray, BH: int, n_pairs: int, slots: int):
     out = {}
     ids = np.arange(costs.size)
@@ -408,6 +456,18 @@ def run_gpu(args):
         dense_ms = e0.elapsed_time(e1) / 3
         del od
 
+    # one traced attention launch (outside the timed region): measured SM-level balance
+    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+    trace = torch.empty((fva.fva_num_tiles(s), 4), dtype=torch.int64, device=dev)
+    fva.fva_set_cta_trace(trace)
+    try:
+        layer.attend()
+        torch.cuda.synchronize()
+    finally:
+        fva.fva_set_cta_trace(None)
+    sm_measured = measured_sm_imbalance(trace.cpu().numpy(), sm_count)
+    del trace
+
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     h2d = 3 * hq.numel() * hq.element_size()
     d2h = ho.numel() * ho.element_size()
@@ -429,8 +489,14 @@ def run_gpu(args):
     if world > 1:
         e2e_ms = ranks_max([e2e_ms], dist, dev)[0]
 
-    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
     imb = imbalance(costs, BH, (nB + 1) // 2, 2 * sm_count)
+    head_bytes = 4.0 * N * d * (2 if wl.dtype == "bf16" else 4)  # Q, K, V in and O out
+    rlb = rlb_report(costs, BH, (nB + 1) // 2, t_attn, head_bytes)
+    if len(per_step) > 1:
+        rlb["per_step"] = []
+        for x in per_step:
+            r = rlb_report(x[2], BH, (nB + 1) // 2, t_attn, head_bytes)
+            rlb["per_step"].append({"before": r["before"], "after": r["after"], "moves": len(r["moves"])})
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -472,6 +538,8 @@ def run_gpu(args):
                          "kernel": "attn_bf16_kernel (fva_sparse_attn)",
                          "peak_source": f"{how} bf16_tflops_sustained (kernel timed inside a multi-second loop)"},
             "imbalance_sm_slots": imb,
+            "imbalance_sm_measured": sm_measured,
+            "rlb_virtual_ranks": rlb,
             "e2e": {"value": round(e2e_ms, 3), "unit": "ms/layer", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h)},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,

@@ -124,6 +124,20 @@ FVA_API int fva_version(void);
 enum { FVA_DIAG_WITHHOLD_Q = 1 };
 FVA_API void fva_set_diagnostics(uint64_t wait_limit_ns, int flags);
 
+/*
+ * Per-CTA trace of the attention kernels (measurement aid; the pages have no
+ * counterpart). While set, every bf16 fva_sparse_attn / fva_dense_attn launch (the
+ * tensor-core kernel; fp32 inputs are not traced) has each CTA write four int64 at
+ * trace_dev[4 * c ..] for CTA (tile launch slot) c:
+ *   [0] the SM it ran on (%smid), [1] its list length in 64-key blocks,
+ *   [2] %globaltimer (ns) when it started, [3] %globaltimer when it finished.
+ * trace_dev: device memory owned by the caller, capacity_ctas * 4 int64, 8-byte aligned;
+ * slot c of a sparse launch is the c-th tile of the work list. A launch with more CTAs
+ * than capacity_ctas fails with FVA_ERR_CAPACITY before launching.
+ * fva_set_cta_trace(NULL, 0) turns tracing off (the default). Process-wide setting; not
+ * thread-safe against concurrent launches. Returns FVA_OK or FVA_ERR_INVALID_ARG. */
+FVA_API int fva_set_cta_trace(int64_t* trace_dev, int64_t capacity_ctas);
+
 /* Derived sizes; -1 for an invalid shape. */
 FVA_API int64_t fva_num_tokens(const fva_shape* s);
 FVA_API int64_t fva_num_blocks(const fva_shape* s);
@@ -246,6 +260,36 @@ FVA_API int fva_dense_attn(const fva_shape* s, const void* q_dev, const void* k_
 FVA_API int fva_route_noalloc(const fva_shape* s, const void* q_bhnd_dev, const void* k_bhnd_dev,
                               const double* pooled_q_dev, const double* pooled_k_dev, double p, int k_floor,
                               int order, const fva_mask* mask, int32_t* dev_status, fva_stream_t stream);
+
+/*
+ * Runtime Load Balancing planner (host code; [aixai] "Runtime Load Balancing (RLB)", [PD]
+ * 方法揭秘). Plans head migrations for a virtual n_ranks-way head split of the measured
+ * per-head loads: heads start in the contiguous split (rank r owns heads
+ * [r * n_heads / n_ranks, (r + 1) * n_heads / n_ranks)); while the slowest / fastest rank
+ * load ratio is >= threshold, the heaviest own head of the most loaded rank whose move to
+ * the least loaded rank has positive net gain G = K - P - C is moved there, where
+ * K = (max rank load before - max after) and P = comm_ms, C = sched_ms; a rank exports at
+ * most max_per_rank of its own heads, and received heads never move again. Ties go to the
+ * lower rank / head index.
+ *   head_load_ms: host double[n_heads], >= 0 (per-head compute time, e.g. blocks x c);
+ *   rank_of_out: host int32[n_heads], the final rank of every head;
+ *   moves_out: host array of moves_capacity records, filled in the order applied;
+ *     moves_capacity must be >= min(n_heads, n_ranks * max_per_rank) (FVA_ERR_CAPACITY);
+ *   n_moves_out: number of records written.
+ * threshold >= 1 (the pages' regime boundary k2 = 1.10 is the usual value). Returns FVA_OK,
+ * FVA_ERR_INVALID_ARG or FVA_ERR_CAPACITY; enqueues no device work.
+ */
+typedef struct {
+  int32_t head;
+  int32_t from_rank;
+  int32_t to_rank;
+  int32_t reserved;
+  double gain_ms; /* net gain G of this move */
+} fva_rlb_move;
+
+FVA_API int fva_rlb_plan(const double* head_load_ms, int n_heads, int n_ranks, double comm_ms, double sched_ms,
+                         double threshold, int max_per_rank, int32_t* rank_of_out, fva_rlb_move* moves_out,
+                         int moves_capacity, int* n_moves_out);
 
 #ifdef __cplusplus
 }

@@ -112,3 +112,17 @@ def test_host_validation_before_any_launch():
     # fp16 conversion is a forward reorder of bf16 data only
     assert fva.call_raw("fva_reorder", ctypes.byref(s), one, P(48), None, one, fva.FVA_FWD_F16, None) == \
         fva.FVA_ERR_INVALID_ARG
+
+
+def test_cta_trace_argument_checks():
+    # host-side checks only; the pointers below are never dereferenced, and tracing is
+    # switched off again before the test ends
+    L = fva.lib()
+    try:
+        assert L.fva_set_cta_trace(None, 5) == fva.FVA_ERR_INVALID_ARG
+        assert L.fva_set_cta_trace(1024, 0) == fva.FVA_ERR_INVALID_ARG
+        assert L.fva_set_cta_trace(1024, -1) == fva.FVA_ERR_INVALID_ARG
+        assert L.fva_set_cta_trace(1028, 4) == fva.FVA_ERR_ALIGNMENT
+        assert L.fva_set_cta_trace(1024, 4) == fva.FVA_OK
+    finally:
+        assert L.fva_set_cta_trace(None, 0) == fva.FVA_OK

@@ -1,0 +1,42 @@
+"""Host-side reductions of bench.py checked on hand-made inputs (no GPU)."""
+import numpy as np
+import pytest
+
+import bench
+
+
+def test_measured_sm_imbalance_hand_trace():
+    # 3 SMs; SM 0 runs two CTAs (10 + 30 blocks), SM 1 one (20), SM 2 none
+    ms = 1_000_000  # ns
+    tr = np.array([[0, 10, 100 * ms, 200 * ms],
+                   [1, 20, 100 * ms, 300 * ms],
+                   [0, 30, 150 * ms, 500 * ms]], dtype=np.int64)
+    r = bench.measured_sm_imbalance(tr, 3)
+    assert r["ctas"] == 3 and r["sms"] == 3
+    # work per SM = 40, 20, 0 -> max/mean = 40 / 20
+    assert r["sm_work_max_over_mean"] == pytest.approx(2.0)
+    assert r["sm_work_max_over_min"] == pytest.approx(40.0)  # empty SM counted as 1 block
+    # span = 500 - 100 = 400 ms; finish = 400, 200, 0 -> mean 200
+    assert r["span_ms"] == pytest.approx(400.0)
+    assert r["sm_finish_mean_over_span"] == pytest.approx(0.5)
+
+
+def test_measured_sm_imbalance_balanced():
+    rng = np.random.default_rng(3)
+    sms = 8
+    tr = np.stack([np.arange(64) % sms, np.full(64, 7), rng.integers(0, 10, 64), np.full(64, 1000)], 1)
+    r = bench.measured_sm_imbalance(tr.astype(np.int64), sms)
+    assert r["sm_work_max_over_mean"] == pytest.approx(1.0)
+    assert r["sm_work_max_over_min"] == pytest.approx(1.0)
+    assert r["sm_finish_mean_over_span"] == pytest.approx(1.0)
+
+
+def test_rlb_report_on_hand_costs():
+    # 4 heads x 2 tiles; head loads in tile steps 18, 2, 2, 2 -> ranks (2 ranks) 20 | 4
+    costs = np.array([9, 9, 1, 1, 1, 1, 1, 1], dtype=np.int64)
+    r = bench.rlb_report(costs, 4, 2, t_attn_ms=24.0, head_bytes=0.0, ranks=2)  # 1 ms per tile step
+    assert r["before"]["makespan_ms"] == pytest.approx(20.0)
+    assert r["before"]["max_over_min"] == pytest.approx(5.0)
+    # moving head 0 (18) would overshoot; head 1 (2) gives 18 | 6
+    assert r["moves"] == [[1, 0, 1]]
+    assert r["after"]["makespan_ms"] == pytest.approx(18.0)
