@@ -144,6 +144,16 @@ int fva_hilbert_perm(const fva_shape* s, int32_t* perm_dev, int32_t* inv_dev, fv
   return cuda_status(launch_hilbert_perm(D, s->T, s->Hg, s->Wg, perm_dev, inv_dev, stream));
 }
 
+int fva_curve_perm(const fva_shape* s, int curve, int32_t* perm_dev, int32_t* inv_dev, int32_t* dev_status,
+                   fva_stream_t stream) {
+  Dims D;
+  if (!s || !perm_dev || !inv_dev) return FVA_ERR_INVALID_ARG;
+  if (curve != FVA_CURVE_HILBERT && curve != FVA_CURVE_RECT) return FVA_ERR_INVALID_ARG;
+  if (!make_dims(s, &D)) return FVA_ERR_UNSUPPORTED_SHAPE;
+  if (curve == FVA_CURVE_HILBERT) return cuda_status(launch_hilbert_perm(D, s->T, s->Hg, s->Wg, perm_dev, inv_dev, stream));
+  return cuda_status(launch_rect_curve_perm(D, s->Hg, s->Wg, perm_dev, inv_dev, dev_status, stream));
+}
+
 int fva_reorder(const fva_shape* s, const void* x_in_dev, void* x_out_dev, double* pooled_dev,
                 const int32_t* perm_dev, int direction, fva_stream_t stream) {
   Dims D;

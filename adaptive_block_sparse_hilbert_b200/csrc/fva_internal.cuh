@@ -29,6 +29,8 @@ __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a -
 // ---------------------------------------------------------------------------------
 cudaError_t launch_hilbert_perm(const Dims& D, int T, int Hg, int Wg, int32_t* perm, int32_t* inv,
                                 cudaStream_t st);
+cudaError_t launch_rect_curve_perm(const Dims& D, int Hg, int Wg, int32_t* perm, int32_t* inv,
+                                   int32_t* dev_status, cudaStream_t st);
 cudaError_t launch_reorder(const Dims& D, const void* x_in, void* x_out, double* pooled,
                            const int32_t* perm, int direction, cudaStream_t st);
 cudaError_t launch_pool(const Dims& D, const void* x_bhnd, double* pooled, cudaStream_t st);

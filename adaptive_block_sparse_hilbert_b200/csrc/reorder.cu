@@ -86,6 +86,78 @@ __global__ void hilbert_frames_kernel(int64_t HW, int64_t N, int32_t* perm, int3
   }
 }
 
+// Generalized Hilbert curve over the Hg x Wg frame itself (J. Cerveny's construction): a
+// region (first cell, major vector a, minor vector b) one cell thick is walked straight;
+// one at least 1.5x longer than thick is cut across a into two halves; otherwise it is cut
+// into three parts (half of b first with the roles of a and b swapped, the far part of b,
+// then back along -b). Halves are rounded to even lengths so the pieces join by unit
+// steps. One thread walks the frame with an explicit stack of pending regions; a stack
+// that would overflow, or a cell count other than Hg * Wg, is reported, never written past.
+struct RectRegion {
+  int x, y, ax, ay, bx, by;
+};
+constexpr int kRectStack = 256;
+
+__device__ __forceinline__ int isign(int v) { return (v > 0) - (v < 0); }
+
+__global__ void rect_curve_frame_kernel(int Hg, int Wg, int32_t* perm, int32_t* dev_status) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  RectRegion stack[kRectStack];
+  int top = 0;
+  stack[top++] = Wg >= Hg ? RectRegion{0, 0, Wg, 0, 0, Hg} : RectRegion{0, 0, 0, Hg, Wg, 0};
+  const int total = Hg * Wg;
+  int n = 0;
+  while (top > 0) {
+    const RectRegion r = stack[--top];
+    const int w = abs(r.ax + r.ay), h = abs(r.bx + r.by);
+    const int ux = isign(r.ax), uy = isign(r.ay), vx = isign(r.bx), vy = isign(r.by);
+    if (h == 1 || w == 1) {
+      const int len = h == 1 ? w : h;
+      const int sx = h == 1 ? ux : vx, sy = h == 1 ? uy : vy;
+      for (int i = 0; i < len; ++i) {
+        const int cx = r.x + i * sx, cy = r.y + i * sy;
+        if (n >= total || cx < 0 || cx >= Wg || cy < 0 || cy >= Hg) {
+          report(dev_status, FVA_DEVERR_MASK);
+          return;
+        }
+        perm[n++] = cy * Wg + cx;
+      }
+      continue;
+    }
+    if (top + 3 > kRectStack) {
+      report(dev_status, FVA_DEVERR_MASK);
+      return;
+    }
+    int na = w / 2, nb = h / 2;
+    if (2 * w > 3 * h) {
+      if ((na & 1) && w > 2) ++na;
+      // children pushed last-first so the first one is walked next
+      stack[top++] = RectRegion{r.x + ux * na, r.y + uy * na, r.ax - ux * na, r.ay - uy * na, r.bx, r.by};
+      stack[top++] = RectRegion{r.x, r.y, ux * na, uy * na, r.bx, r.by};
+    } else {
+      if ((nb & 1) && h > 2) ++nb;
+      const int a2x = ux * na, a2y = uy * na, b2x = vx * nb, b2y = vy * nb;
+      stack[top++] = RectRegion{r.x + (r.ax - ux) + (b2x - vx), r.y + (r.ay - uy) + (b2y - vy), -b2x, -b2y,
+                                -(r.ax - a2x), -(r.ay - a2y)};
+      stack[top++] = RectRegion{r.x + b2x, r.y + b2y, r.ax, r.ay, r.bx - b2x, r.by - b2y};
+      stack[top++] = RectRegion{r.x, r.y, b2x, b2y, a2x, a2y};
+    }
+  }
+  if (n != total) report(dev_status, FVA_DEVERR_MASK);
+}
+
+cudaError_t launch_rect_curve_perm(const Dims& D, int Hg, int Wg, int32_t* perm, int32_t* inv,
+                                   int32_t* dev_status, cudaStream_t st) {
+  rect_curve_frame_kernel<<<1, 32, 0, st>>>(Hg, Wg, perm, dev_status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t HW = static_cast<int64_t>(Hg) * Wg;
+  int grid = static_cast<int>((D.N + 255) / 256);
+  if (grid > 148 * 16) grid = 148 * 16;
+  hilbert_frames_kernel<<<grid, 256, 0, st>>>(HW, D.N, perm, inv);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_hilbert_perm(const Dims& D, int T, int Hg, int Wg, int32_t* perm, int32_t* inv,
                                 cudaStream_t st) {
   int m = 0;

@@ -92,6 +92,7 @@ def _load():
         "fva_route_workspace_bytes": (sz, [S, i32]),
         "fva_tiles_workspace_bytes": (sz, [S]),
         "fva_hilbert_perm": (i32, [S, P, P, P]),
+        "fva_curve_perm": (i32, [S, i32, P, P, P, P]),
         "fva_reorder": (i32, [S, P, P, P, P, i32, P]),
         "fva_pool": (i32, [S, P, P, P]),
         "fva_route": (i32, [S, P, P, P, P, dbl, i32, i32, M, P, sz, P, P]),
@@ -112,7 +113,7 @@ EXPORTED = (
     "fva_status_string", "fva_version", "fva_set_diagnostics", "fva_num_tokens", "fva_num_blocks", "fva_num_tiles", "fva_mask_capacity",
     "fva_tile_capacity", "fva_route_workspace_bytes", "fva_tiles_workspace_bytes", "fva_hilbert_perm", "fva_reorder",
     "fva_pool", "fva_route", "fva_build_tiles", "fva_sparse_attn", "fva_dense_attn", "fva_route_noalloc",
-    "fva_set_cta_trace", "fva_rlb_plan",
+    "fva_set_cta_trace", "fva_rlb_plan", "fva_curve_perm",
 )
 
 
@@ -242,6 +243,15 @@ class Mask:
 
 def fva_hilbert_perm(s, perm, inv, stream=None):
     _check("fva_hilbert_perm", _lib.fva_hilbert_perm(ctypes.byref(s), _ptr(perm), _ptr(inv), _stream(stream)))
+
+
+FVA_CURVE_HILBERT = 0
+FVA_CURVE_RECT = 1
+
+
+def fva_curve_perm(s, curve, perm, inv, dev_status=None, stream=None):
+    _check("fva_curve_perm", _lib.fva_curve_perm(ctypes.byref(s), int(curve), _ptr(perm), _ptr(inv), _ptr(dev_status),
+                                                 _stream(stream)))
 
 
 def fva_reorder(s, x_in, x_out, pooled, perm, direction=FVA_FWD, stream=None):

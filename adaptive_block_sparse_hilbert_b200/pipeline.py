@@ -14,7 +14,7 @@ from . import fva
 
 class SparseAttentionLayer:
     def __init__(self, shape: fva.fva_shape, p: float, k_floor: int, order: int = fva.FVA_ORDER_HEAD_LPT,
-                 device: str = "cuda", v_fp16: bool = True):
+                 device: str = "cuda", v_fp16: bool = True, curve: int = fva.FVA_CURVE_HILBERT):
         self.shape = shape
         self.p = float(p)
         self.k_floor = int(k_floor)
@@ -40,7 +40,8 @@ class SparseAttentionLayer:
         ws = fva.fva_route_workspace_bytes(s, False)
         self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
         self.dev_status = torch.zeros(1, dtype=torch.int32, device=device)
-        fva.fva_hilbert_perm(s, self.perm, self.inv)
+        self.curve = int(curve)
+        fva.fva_curve_perm(s, self.curve, self.perm, self.inv, self.dev_status)
 
     def reorder_inputs(self, q, k, v, stream=None):
         s = self.shape

@@ -339,7 +339,8 @@ def run_gpu(args):
     qkv_steps = [(q, k, v)] + [tuple(host(a, b).to(dev) for a, b in ((X.q, X.q_bits), (X.k, X.k_bits), (X.v, X.v_bits)))
                                for X in layers_np[1:]]
     o = torch.empty_like(q)
-    layer = pipeline.SparseAttentionLayer(s, wl.p, wl.k_floor, device=dev)
+    curve = fva.FVA_CURVE_RECT if args.curve == "rect" else fva.FVA_CURVE_HILBERT
+    layer = pipeline.SparseAttentionLayer(s, wl.p, wl.k_floor, device=dev, curve=curve)
     stream = torch.cuda.current_stream()
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
@@ -520,7 +521,7 @@ def run_gpu(args):
             "dtype": "bf16" if wl.dtype == "bf16" else "f32",
             "data": "synthetic",
             "config": {"workload": wl.name, "tokens": N, "grid": [wl.T, wl.Hg, wl.Wg], "heads": wl.H,
-                       "head_dim": d, "block": 64, "p": wl.p, "k_floor": wl.k_floor, "order": "head_lpt",
+                       "head_dim": d, "block": 64, "p": wl.p, "k_floor": wl.k_floor, "order": "head_lpt", "curve": args.curve,
                        "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (3 x %.0f MB)" % (q.numel() * q.element_size() / 1e6)},
             "kept_tflops": round(achieved_tf, 1),
@@ -564,6 +565,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", type=int, default=2)
     ap.add_argument("--p", type=float, default=None)
+    ap.add_argument("--curve", default="hilbert", choices=["hilbert", "rect"],
+                    help="token order: Hilbert curve on the enclosing 2^m square (the pages' reading) or the "
+                         "generalized Hilbert curve over the frame itself")
     ap.add_argument("--impl", default="fva", choices=["fva", "reference"])
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

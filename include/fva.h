@@ -159,6 +159,22 @@ FVA_API size_t fva_route_workspace_bytes(const fva_shape* s, int need_pool);
 FVA_API int fva_hilbert_perm(const fva_shape* s, int32_t* perm_dev, int32_t* inv_dev, fva_stream_t stream);
 
 /*
+ * Token order by a chosen curve. FVA_CURVE_HILBERT is fva_hilbert_perm's order.
+ * FVA_CURVE_RECT is a variant the pages leave open: a generalized Hilbert curve laid over
+ * the Hg x Wg frame itself (J. Cerveny's construction: rectangles cut along the long side
+ * into two halves, or across it into three parts, halves rounded to even lengths), which
+ * keeps every step between grid neighbours where the plain curve on the enclosing 2^m
+ * square jumps over skipped cells; on 2^m x 2^m frames the two orders are equal. The
+ * curve starts at (x, y) = (0, 0) and runs first along the longer side. perm_dev / inv_dev
+ * as for fva_hilbert_perm; dev_status (optional) receives FVA_DEVERR_MASK if the walk
+ * fails its own consistency checks. Returns FVA_OK, FVA_ERR_INVALID_ARG (unknown curve),
+ * FVA_ERR_UNSUPPORTED_SHAPE or FVA_ERR_CUDA.
+ */
+enum { FVA_CURVE_HILBERT = 0, FVA_CURVE_RECT = 1 };
+FVA_API int fva_curve_perm(const fva_shape* s, int curve, int32_t* perm_dev, int32_t* inv_dev, int32_t* dev_status,
+                           fva_stream_t stream);
+
+/*
  * Token reorder with fused block mean-pooling ([aixai] "Sparse-routing frontend"; [PD]
  * 方法揭秘: block importance from pooled Q/K).
  *   FVA_FWD: x_out[b, h, i, :] = x_in[b, perm[i], h, :]   ([B,N,H,d] -> [B,H,N,d]);

@@ -99,6 +99,69 @@ def hilbert_perm(T: int, Hg: int, Wg: int):
     return perm, inv
 
 
+# Variant of step 1 (a next step of the build, not the pages' own): a generalized
+# Hilbert curve that covers a W x H rectangle directly instead of the enclosing 2^m
+# square, following Jakub Cerveny's published generalized-Hilbert ("gilbert")
+# construction: a rectangle is split along its longer side into two halves, or across
+# it into three parts whose middle part runs the other way, with half lengths rounded to
+# even so that the pieces join by unit steps. On 2^m squares it is the curve above.
+
+
+def rect_hilbert_curve(W: int, H: int) -> np.ndarray:
+    """Cells of the W x H rectangle in generalized-Hilbert visiting order, int [W*H, 2] of (x, y).
+
+    A region is given by its first cell (x, y), a major vector a (along which the curve
+    leaves the region) and a minor vector b, both axis-parallel. A region one cell thick
+    is walked straight. A region at least 1.5 times longer than thick is cut across a into
+    two regions with the same a direction. Otherwise it is cut into three: a first region
+    whose major vector is the first half of b (and minor vector the first half of a), the
+    far part along b with the original vectors, and a last region that returns along -b.
+    """
+    cells = []
+
+    def sign(v):
+        return (v > 0) - (v < 0)
+
+    def region(x, y, ax, ay, bx, by):
+        w, h = abs(ax + ay), abs(bx + by)
+        ux, uy, vx, vy = sign(ax), sign(ay), sign(bx), sign(by)
+        if h == 1:
+            cells.extend((x + i * ux, y + i * uy) for i in range(w))
+            return
+        if w == 1:
+            cells.extend((x + i * vx, y + i * vy) for i in range(h))
+            return
+        na, nb = w // 2, h // 2
+        if 2 * w > 3 * h:
+            if na % 2 == 1 and w > 2:
+                na += 1
+            region(x, y, ux * na, uy * na, bx, by)
+            region(x + ux * na, y + uy * na, ax - ux * na, ay - uy * na, bx, by)
+        else:
+            if nb % 2 == 1 and h > 2:
+                nb += 1
+            a2x, a2y, b2x, b2y = ux * na, uy * na, vx * nb, vy * nb
+            region(x, y, b2x, b2y, a2x, a2y)
+            region(x + b2x, y + b2y, ax, ay, bx - b2x, by - b2y)
+            region(x + (ax - ux) + (b2x - vx), y + (ay - uy) + (b2y - vy), -b2x, -b2y, -(ax - a2x), -(ay - a2y))
+
+    if W >= H:
+        region(0, 0, W, 0, 0, H)
+    else:
+        region(0, 0, 0, H, W, 0)
+    return np.array(cells, dtype=np.int64).reshape(-1, 2)
+
+
+def rect_curve_perm(T: int, Hg: int, Wg: int):
+    """As ``hilbert_perm`` with the frame order of ``rect_hilbert_curve(Wg, Hg)``."""
+    frame = np.array([y * Wg + x for (x, y) in rect_hilbert_curve(Wg, Hg)], dtype=np.int64)
+    hw = Hg * Wg
+    perm = np.concatenate([t * hw + frame for t in range(T)]) if T > 0 else np.zeros(0, np.int64)
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(perm.size, dtype=np.int64)
+    return perm, inv
+
+
 def reorder(x_bnhd: np.ndarray, perm: np.ndarray) -> np.ndarray:
     """[B, N, H, d] raster -> [B, H, N, d] Hilbert order: out[b, h, i] = x[b, perm[i], h] (float64)."""
     x = np.asarray(x_bnhd, dtype=np.float64)

@@ -46,7 +46,7 @@ def to_device(L):
 class GpuRun:
     """Runs the CUDA path step by step and keeps every intermediate (on the device)."""
 
-    def __init__(self, wl, L, p=None, k_floor=None, order=None, need_pool=False):
+    def __init__(self, wl, L, p=None, k_floor=None, order=None, need_pool=False, curve=None):
         torch = torch_dev()
         from adaptive_block_sparse_hilbert_b200 import fva, pipeline
         self.fva = fva
@@ -56,6 +56,8 @@ class GpuRun:
         kw = {}
         if order is not None:
             kw["order"] = order
+        if curve is not None:
+            kw["curve"] = curve
         self.layer = pipeline.SparseAttentionLayer(s, wl.p if p is None else p,
                                                    wl.k_floor if k_floor is None else k_floor, **kw)
         self.q, self.k, self.v = to_device(L)

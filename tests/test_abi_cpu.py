@@ -126,3 +126,9 @@ def test_cta_trace_argument_checks():
         assert L.fva_set_cta_trace(1024, 4) == fva.FVA_OK
     finally:
         assert L.fva_set_cta_trace(None, 0) == fva.FVA_OK
+
+
+def test_curve_perm_rejects_unknown_curve():
+    s = fva.make_shape(1, 1, 64, 2, 8, 8, "bf16")
+    assert fva.lib().fva_curve_perm(ctypes.byref(s), 7, 1024, 2048, None, None) == fva.FVA_ERR_INVALID_ARG
+    assert fva.lib().fva_curve_perm(ctypes.byref(s), fva.FVA_CURVE_RECT, None, 2048, None, None) == fva.FVA_ERR_INVALID_ARG

@@ -31,6 +31,27 @@ def test_hilbert_perm_exact(T, Hg, Wg):
     np.testing.assert_array_equal(inv.cpu().numpy(), want_i)
 
 
+@pytest.mark.parametrize("T,Hg,Wg", GRIDS + [(1, 40, 40), (2, 1, 77), (3, 33, 17)])
+def test_rect_curve_perm_exact(T, Hg, Wg):
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import fva
+    s = fva.make_shape(1, 1, 64, T, Hg, Wg, "bf16")
+    N = T * Hg * Wg
+    perm = torch.empty(N, dtype=torch.int32, device="cuda")
+    inv = torch.empty(N, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fva.fva_curve_perm(s, fva.FVA_CURVE_RECT, perm, inv, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    want_p, want_i = O.rect_curve_perm(T, Hg, Wg)
+    np.testing.assert_array_equal(perm.cpu().numpy(), want_p)
+    np.testing.assert_array_equal(inv.cpu().numpy(), want_i)
+    # the plain curve through the same entry point is fva_hilbert_perm's order
+    fva.fva_curve_perm(s, fva.FVA_CURVE_HILBERT, perm, inv, st)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(perm.cpu().numpy(), O.hilbert_perm(T, Hg, Wg)[0])
+
+
 SMALL = [
     synth.WORKLOADS[0],
     synth.custom_workload(3, 10, 13, 3, 64, "bf16", seed=11),    # N = 390, tail block of 6

@@ -15,17 +15,17 @@ from tests import _common as C
 pytestmark = pytest.mark.gpu
 
 
-def _oracle_mask(wl, L, p, k_floor):
-    perm, _ = O.hilbert_perm(wl.T, wl.Hg, wl.Wg)
+def _oracle_mask(wl, L, p, k_floor, curve=0):
+    perm, _ = (O.rect_curve_perm if curve == 1 else O.hilbert_perm)(wl.T, wl.Hg, wl.Wg)
     pq, pk = C.oracle_pooled(L, perm)
     return O.route(pq, pk, wl.d, p, k_floor, with_ambiguity=True)
 
 
-def _check_route(wl, L, p, k_floor, order=2, need_pool=False, max_amb_frac=2e-2):
-    run = C.GpuRun(wl, L, p=p, k_floor=k_floor, order=order, need_pool=need_pool)
+def _check_route(wl, L, p, k_floor, order=2, need_pool=False, max_amb_frac=2e-2, curve=None):
+    run = C.GpuRun(wl, L, p=p, k_floor=k_floor, order=order, need_pool=need_pool, curve=curve)
     assert run.status() == 0
     g = run.mask_np()
-    o = _oracle_mask(wl, L, p, k_floor)
+    o = _oracle_mask(wl, L, p, k_floor, curve or 0)
     BH, nB = wl.B * wl.H, wl.nB
     mism, amb = C.compare_masks(g, o, BH * nB)
     n_amb = int(amb.sum())
@@ -149,3 +149,10 @@ def test_hetero_heads_density_split():
     print(f"flat-head share of kept blocks: {share:.3f}")
     assert hk[flat].min() > 2 * hk[~flat].max()
     assert share > 0.3
+
+
+@pytest.mark.parametrize("wid", [1, 3, 2])
+def test_route_full_size_rect_curve(wid):
+    """The same acceptance with tokens ordered by the generalized (rectangular) Hilbert curve."""
+    wl = synth.WORKLOADS[wid]
+    _check_route(wl, C.layer(wid), wl.p, wl.k_floor, order=2, curve=1)
