@@ -222,6 +222,50 @@ int fva_route(const fva_shape* s, const void* q_bhnd_dev, const void* k_bhnd_dev
   return cuda_status(launch_route(D, pq, pk, p, k_floor, order, mask, rs, dev_status, stream));
 }
 
+size_t fva_sasa_workspace_bytes(const fva_shape* s) {
+  Dims D;
+  if (!make_dims(s, &D)) return 0;
+  return route_scratch_layout(D, 0, nullptr, nullptr, nullptr, nullptr, true) + sasa_extra_bytes(D);
+}
+
+int fva_sasa_augment(const fva_shape* s, const double* pooled_q_dev, const double* pooled_k_dev,
+                     const int32_t* rank_of_head_dev, int n_ranks, const int64_t* budget_dev, int order,
+                     const fva_mask* mask, void* workspace_dev, size_t workspace_bytes, int64_t* added_dev,
+                     int32_t* dev_status, fva_stream_t stream) {
+  Dims D;
+  if (!s || !pooled_q_dev || !pooled_k_dev || !rank_of_head_dev || !budget_dev || !workspace_dev)
+    return FVA_ERR_INVALID_ARG;
+  if (n_ranks < 1 || n_ranks > FVA_SASA_MAX_RANKS) return FVA_ERR_INVALID_ARG;
+  if (order != FVA_ORDER_NATURAL && order != FVA_ORDER_LPT && order != FVA_ORDER_HEAD_LPT) return FVA_ERR_INVALID_ARG;
+  if (!make_dims(s, &D)) return FVA_ERR_UNSUPPORTED_SHAPE;
+  if (!route_shape_supported(D)) return FVA_ERR_UNSUPPORTED_SHAPE;
+  int rc = check_mask_outputs(D, mask);
+  if (rc != FVA_OK) return rc;
+  const size_t base = route_scratch_layout(D, 0, nullptr, nullptr, nullptr, nullptr, true);
+  if (workspace_bytes < base + sasa_extra_bytes(D)) return FVA_ERR_WORKSPACE;
+  if (!aligned16(workspace_dev) || !aligned16(pooled_q_dev) || !aligned16(pooled_k_dev)) return FVA_ERR_ALIGNMENT;
+  RouteScratch rs;
+  route_scratch_layout(D, 0, workspace_dev, &rs, nullptr, nullptr, true);
+  return cuda_status(launch_sasa(D, pooled_q_dev, pooled_k_dev, rank_of_head_dev, n_ranks, budget_dev, order, mask,
+                                 rs, static_cast<uint8_t*>(workspace_dev) + base, added_dev, dev_status, stream));
+}
+
+int fva_sasa_budgets(const double* rank_load_ms, int n_ranks, double block_ms, double n1, double n2,
+                     int64_t* budget_out) {
+  if (!rank_load_ms || !budget_out || n_ranks < 1) return FVA_ERR_INVALID_ARG;
+  if (!(block_ms > 0.0) || !(n1 >= 0.0) || !(n2 >= 0.0)) return FVA_ERR_INVALID_ARG;
+  double crit = 0.0;
+  for (int r = 0; r < n_ranks; ++r) {
+    if (!(rank_load_ms[r] >= 0.0) || isinf(rank_load_ms[r])) return FVA_ERR_INVALID_ARG;
+    if (rank_load_ms[r] > crit) crit = rank_load_ms[r];
+  }
+  for (int r = 0; r < n_ranks; ++r) {
+    const double slack = crit - rank_load_ms[r];
+    budget_out[r] = (crit > 0.0 && slack >= n2 * crit) ? static_cast<int64_t>(floor(n1 * slack / block_ms)) : 0;
+  }
+  return FVA_OK;
+}
+
 int fva_build_tiles(const fva_shape* s, const fva_mask* mask, int order, void* workspace_dev, size_t workspace_bytes,
                     int32_t* dev_status, fva_stream_t stream) {
   Dims D;

@@ -46,6 +46,15 @@ cudaError_t launch_route(const Dims& D, const double* pq, const double* pk, doub
                          cudaStream_t st);
 cudaError_t launch_build_tiles(const Dims& D, const fva_mask* m, int order, const RouteScratch& ws,
                                int32_t* dev_status, cudaStream_t st);
+size_t sasa_extra_bytes(const Dims& D);
+cudaError_t launch_sasa(const Dims& D, const double* pq, const double* pk, const int32_t* rank_of, int R,
+                        const int64_t* budget, int order, const fva_mask* m, const RouteScratch& ws, uint8_t* extra,
+                        int64_t* added, int32_t* dev_status, cudaStream_t st);
+cudaError_t launch_route_scores(const Dims& D, const double* pq, const double* pk, double* scores, cudaStream_t st);
+cudaError_t launch_csr_to_bits(const Dims& D, const fva_mask* m, uint32_t* bits, int32_t* dev_status,
+                               cudaStream_t st);
+cudaError_t launch_tiles_from_bits(const Dims& D, const fva_mask* m, int order, const RouteScratch& ws,
+                                   const int32_t* row_cnt, int write_rows, int32_t* dev_status, cudaStream_t st);
 
 cudaError_t launch_attn_bf16(const Dims& D, const void* q, const void* k, const void* v, bool v_f16,
                              const fva_mask* m, bool dense, void* o, float scale,

@@ -680,10 +680,7 @@ cudaError_t launch_route(const Dims& D, const double* pq, const double* pk, doub
                          const fva_mask* m, const RouteScratch& ws, int32_t* dev_status, cudaStream_t st) {
   const int nB = static_cast<int>(D.nB);
   {
-    const dim3 grid((nB + kST - 1) / kST, (nB + kST - 1) / kST, static_cast<unsigned>(D.BH));
-    route_scores_kernel<<<grid, 256, 0, st>>>(pq, pk, ws.scores, nB, static_cast<int>(D.d),
-                                              sqrt(static_cast<double>(D.d)));
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_route_scores(D, pq, pk, ws.scores, st);
     if (e != cudaSuccess) return e;
   }
   {
@@ -705,22 +702,42 @@ cudaError_t launch_route(const Dims& D, const double* pq, const double* pk, doub
   return launch_order_and_emit(D, m, order, ws, 1, st);
 }
 
-cudaError_t launch_build_tiles(const Dims& D, const fva_mask* m, int order, const RouteScratch& ws,
-                               int32_t* dev_status, cudaStream_t st) {
+cudaError_t launch_route_scores(const Dims& D, const double* pq, const double* pk, double* scores, cudaStream_t st) {
+  const int nB = static_cast<int>(D.nB);
+  const dim3 grid((nB + kST - 1) / kST, (nB + kST - 1) / kST, static_cast<unsigned>(D.BH));
+  route_scores_kernel<<<grid, 256, 0, st>>>(pq, pk, scores, nB, static_cast<int>(D.d), sqrt(static_cast<double>(D.d)));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_csr_to_bits(const Dims& D, const fva_mask* m, uint32_t* bits, int32_t* dev_status,
+                               cudaStream_t st) {
   csr_to_bits_kernel<<<static_cast<int>((D.rows + 7) / 8), 256, 0, st>>>(
-      m->row_ptr, m->col_idx, D.rows, static_cast<int>(D.nB), static_cast<int>(D.nWords), ws.bits, dev_status);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+      m->row_ptr, m->col_idx, D.rows, static_cast<int>(D.nB), static_cast<int>(D.nWords), bits, dev_status);
+  return cudaGetLastError();
+}
+
+// From per-row bitmasks in ws.bits: tile costs, row_ptr (from row_cnt, or kept as given
+// when row_cnt is null), tile_ptr, head_kept, the work list, then the lists themselves
+// (col_idx too when write_rows).
+cudaError_t launch_tiles_from_bits(const Dims& D, const fva_mask* m, int order, const RouteScratch& ws,
+                                   const int32_t* row_cnt, int write_rows, int32_t* dev_status, cudaStream_t st) {
   tile_cost_kernel<<<static_cast<int>((D.tiles + 7) / 8), 256, 0, st>>>(
       ws.bits, static_cast<int>(D.nB), static_cast<int>(D.nWords), static_cast<int>(D.nPairs), D.tiles, m->tile_cost);
-  e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  finish_kernel<<<1, 1024, 0, st>>>(nullptr, D.rows, m->tile_cost, D.tiles, static_cast<int>(D.nB),
+  finish_kernel<<<1, 1024, 0, st>>>(row_cnt, D.rows, m->tile_cost, D.tiles, static_cast<int>(D.nB),
                                     static_cast<int>(D.nPairs), static_cast<int>(D.BH), m->row_ptr, m->tile_ptr,
                                     m->head_kept, ws.head_load, m->capacity, m->tile_capacity, dev_status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_order_and_emit(D, m, order, ws, 0, st);
+  return launch_order_and_emit(D, m, order, ws, write_rows, st);
+}
+
+cudaError_t launch_build_tiles(const Dims& D, const fva_mask* m, int order, const RouteScratch& ws,
+                               int32_t* dev_status, cudaStream_t st) {
+  cudaError_t e = launch_csr_to_bits(D, m, ws.bits, dev_status, st);
+  if (e != cudaSuccess) return e;
+  return launch_tiles_from_bits(D, m, order, ws, nullptr, 0, dev_status, st);
 }
 
 bool route_shape_supported(const Dims& D) { return select_rows_per_cta(D) > 0; }

@@ -93,6 +93,9 @@ def _load():
         "fva_tiles_workspace_bytes": (sz, [S]),
         "fva_hilbert_perm": (i32, [S, P, P, P]),
         "fva_curve_perm": (i32, [S, i32, P, P, P, P]),
+        "fva_sasa_budgets": (i32, [ctypes.POINTER(ctypes.c_double), i32, dbl, dbl, dbl, ctypes.POINTER(ctypes.c_int64)]),
+        "fva_sasa_workspace_bytes": (sz, [S]),
+        "fva_sasa_augment": (i32, [S, P, P, P, i32, P, i32, M, P, sz, P, P, P]),
         "fva_reorder": (i32, [S, P, P, P, P, i32, P]),
         "fva_pool": (i32, [S, P, P, P]),
         "fva_route": (i32, [S, P, P, P, P, dbl, i32, i32, M, P, sz, P, P]),
@@ -113,7 +116,8 @@ EXPORTED = (
     "fva_status_string", "fva_version", "fva_set_diagnostics", "fva_num_tokens", "fva_num_blocks", "fva_num_tiles", "fva_mask_capacity",
     "fva_tile_capacity", "fva_route_workspace_bytes", "fva_tiles_workspace_bytes", "fva_hilbert_perm", "fva_reorder",
     "fva_pool", "fva_route", "fva_build_tiles", "fva_sparse_attn", "fva_dense_attn", "fva_route_noalloc",
-    "fva_set_cta_trace", "fva_rlb_plan", "fva_curve_perm",
+    "fva_set_cta_trace", "fva_rlb_plan", "fva_curve_perm", "fva_sasa_budgets", "fva_sasa_workspace_bytes",
+    "fva_sasa_augment",
 )
 
 
@@ -160,6 +164,18 @@ def fva_rlb_plan(head_load_ms, n_ranks: int, comm_ms: float, sched_ms: float, th
     if st != 0:
         raise FvaError("fva_rlb_plan", st)
     return rank_of, [(m.head, m.from_rank, m.to_rank, m.gain_ms) for m in moves[:n.value]]
+
+
+def fva_sasa_budgets(rank_load_ms, block_ms: float, n1: float = 0.8, n2: float = 0.07):
+    """Blocks each rank may add (host): floor(n1 * slack / block_ms) where slack >= n2 * critical."""
+    import numpy as np
+    load = np.ascontiguousarray(rank_load_ms, dtype=np.float64)
+    out = np.zeros(load.shape[0], dtype=np.int64)
+    st = _lib.fva_sasa_budgets(load.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), int(load.shape[0]),
+                               float(block_ms), float(n1), float(n2), out.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)))
+    if st != 0:
+        raise FvaError("fva_sasa_budgets", st)
+    return out
 
 
 def status_string(status: int) -> str:
@@ -280,6 +296,19 @@ def fva_route_noalloc(s, q, k, pooled_q, pooled_k, p, k_floor, mask: Mask, order
     _check("fva_route_noalloc", _lib.fva_route_noalloc(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(pooled_q),
                                                        _ptr(pooled_k), float(p), int(k_floor), int(order),
                                                        ctypes.byref(m), _ptr(dev_status), _stream(stream)))
+
+
+def fva_sasa_workspace_bytes(s): return _lib.fva_sasa_workspace_bytes(ctypes.byref(s))
+
+
+def fva_sasa_augment(s, pooled_q, pooled_k, rank_of_head, budget, mask: Mask, workspace, order=FVA_ORDER_HEAD_LPT,
+                     added=None, dev_status=None, stream=None):
+    """Slack-aware augmentation of a routed mask in place (rank_of_head int32 [B*H] and
+    budget int64 [n_ranks] on the device)."""
+    _check("fva_sasa_augment", _lib.fva_sasa_augment(
+        ctypes.byref(s), _ptr(pooled_q), _ptr(pooled_k), _ptr(rank_of_head), int(budget.shape[0]), _ptr(budget),
+        int(order), ctypes.byref(mask.c()), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(added), _ptr(dev_status), _stream(stream)))
 
 
 def fva_build_tiles(s, mask: Mask, workspace, order=FVA_ORDER_HEAD_LPT, dev_status=None, stream=None):

@@ -181,10 +181,87 @@ def rlb_report(costs: np.ndarray, BH: int, n_pairs: int, t_attn_ms: float, head_
                 "makespan_ms": round(float(Lr.max()), 3)}
 
     home = (np.arange(BH) * ranks) // BH
-    return {"ranks": ranks, "heads": BH, "before": stats(home), "after": stats(rank_of.astype(np.int64)),
-            "moves": [[int(h), int(a), int(b)] for h, a, b, _ in moves],
-            "comm_ms_per_head": round(comm, 4), "sched_ms": round(sched, 4),
-            "note": "virtual split on one GPU; ranks run their heads at this GPU's measured rate"}
+    rep = {"ranks": ranks, "heads": BH, "before": stats(home), "after": stats(rank_of.astype(np.int64)),
+           "moves": [[int(h), int(a), int(b)] for h, a, b, _ in moves],
+           "comm_ms_per_head": round(comm, 4), "sched_ms": round(sched, 4),
+           "note": "virtual split on one GPU; ranks run their heads at this GPU's measured rate"}
+    return rep, {"rank_of": rank_of.astype(np.int64), "home": home, "head_load": load}
+
+
+def sasa_report(layer, s, wl, plan, t_attn_ms: float, kept_blocks: int, dev, stream, ranks: int = 8):
+    """Slack-Aware Sparse Augmentation on the virtual head split RLB planned: budgets from
+    the post-RLB rank loads (c = measured time per kept block), the augmentation itself,
+    attention on the augmented mask, and two quality proxies before / after -- the mean
+    routing importance the kept blocks hold per row, and the relative L2 error of the sparse
+    output against the dense kernel's. Runs after the timed region; the mask is changed."""
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import fva
+    BH, nB, d = wl.B * wl.H, wl.nB, wl.d
+    rank_of, load = plan["rank_of"], plan["head_load"]
+    start_load = np.bincount(plan["home"], weights=load, minlength=ranks)
+    rho0 = float(start_load.max() / start_load.min()) if start_load.min() > 0 else float("inf")
+    mode = "none" if rho0 < 1.05 else ("sasa" if rho0 < 1.10 else "rlb+sasa")
+    placed = rank_of if mode == "rlb+sasa" else plan["home"]
+    rank_load = np.bincount(placed, weights=load, minlength=ranks)
+    c_blk = t_attn_ms / max(kept_blocks, 1)
+    budget = fva.fva_sasa_budgets(rank_load, c_blk) if mode != "none" else np.zeros(ranks, dtype=np.int64)
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    def quality():
+        layer.attend()
+        pq = layer.pooled_q.reshape(BH, nB, d)
+        pk = layer.pooled_k.reshape(BH, nB, d)
+        rp = layer.mask.row_ptr.long()
+        ci = layer.mask.col_idx[: int(rp[-1].item())].long()
+        rows = torch.repeat_interleave(torch.arange(BH * nB, device=dev), rp[1:] - rp[:-1])
+        mass = torch.zeros(BH * nB, dtype=torch.float64, device=dev)
+        for h in range(BH):  # one head at a time: [nB, nB] float64 importances
+            P = torch.softmax(pq[h] @ pk[h].T / float(np.sqrt(d)), dim=1).reshape(-1)
+            sel = (rows >= h * nB) & (rows < (h + 1) * nB)
+            mass.index_add_(0, rows[sel], P[(rows[sel] - h * nB) * nB + ci[sel]])
+        od = torch.empty_like(layer.oh)
+        fva.fva_dense_attn(s, layer.qh, layer.kh, layer.vh, od, 0.0, layer.dev_status)
+        diff = (layer.oh.float() - od.float()).reshape(BH, -1)
+        err = float((diff.norm(dim=1) / od.float().reshape(BH, -1).norm(dim=1)).mean())
+        del od
+        return float(mass.mean()), err
+
+    mass0, err0 = quality()
+    ws = torch.empty(fva.fva_sasa_workspace_bytes(s), dtype=torch.uint8, device=dev)
+    rk = torch.as_tensor(placed.astype(np.int32), device=dev)
+    bd = torch.as_tensor(budget.astype(np.int64), device=dev)
+    added = torch.zeros(ranks, dtype=torch.int64, device=dev)
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    fva.fva_sasa_augment(s, layer.pooled_q, layer.pooled_k, rk, bd, layer.mask, ws, fva.FVA_ORDER_HEAD_LPT, added,
+                         layer.dev_status)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_aug = e0.elapsed_time(e1)
+    added_np = added.cpu().numpy()
+    for _ in range(2):
+        layer.attend()
+    e0.record(stream)
+    for _ in range(3):
+        layer.attend()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_attn_aug = e0.elapsed_time(e1) / 3
+    mass1, err1 = quality()
+    after = rank_load + added_np * c_blk
+    del ws
+    return {"mode": mode, "start_max_over_min": round(rho0, 4), "budget_blocks": budget.tolist(),
+            "added_blocks": added_np.tolist(), "block_ms": round(c_blk, 8),
+            "rank_load_ms": [round(float(x), 3) for x in rank_load],
+            "rank_load_after_ms": [round(float(x), 3) for x in after],
+            "critical_ms": round(float(rank_load.max()), 3),
+            "kept_importance_mean": {"before": round(mass0, 5), "after": round(mass1, 5)},
+            "out_rel_l2_vs_dense": {"before": round(err0, 6), "after": round(err1, 6)},
+            "augment_ms": round(t_aug, 3), "attn_ms_one_gpu_after": round(t_attn_aug, 3),
+            "note": "one GPU runs every rank's heads, so its attention time grows by the added blocks; "
+                    "on the virtual split no rank passes the critical load"}
 
 
 def imbalance(costs: np.ndarray, BH: int, n_pairs: int, slots: int):
@@ -492,12 +569,13 @@ def run_gpu(args):
 
     imb = imbalance(costs, BH, (nB + 1) // 2, 2 * sm_count)
     head_bytes = 4.0 * N * d * (2 if wl.dtype == "bf16" else 4)  # Q, K, V in and O out
-    rlb = rlb_report(costs, BH, (nB + 1) // 2, t_attn, head_bytes)
+    rlb, plan = rlb_report(costs, BH, (nB + 1) // 2, t_attn, head_bytes)
     if len(per_step) > 1:
         rlb["per_step"] = []
         for x in per_step:
-            r = rlb_report(x[2], BH, (nB + 1) // 2, t_attn, head_bytes)
+            r, _ = rlb_report(x[2], BH, (nB + 1) // 2, t_attn, head_bytes)
             rlb["per_step"].append({"before": r["before"], "after": r["after"], "moves": len(r["moves"])})
+    sasa = None if args.no_sasa else sasa_report(layer, s, wl, plan, t_attn, kept, dev, stream)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -541,6 +619,7 @@ def run_gpu(args):
             "imbalance_sm_slots": imb,
             "imbalance_sm_measured": sm_measured,
             "rlb_virtual_ranks": rlb,
+            "sasa_virtual_ranks": sasa,
             "e2e": {"value": round(e2e_ms, 3), "unit": "ms/layer", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h)},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
@@ -571,6 +650,7 @@ def main():
     ap.add_argument("--impl", default="fva", choices=["fva", "reference"])
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sasa", action="store_true", help="skip the slack-aware augmentation report")
     ap.add_argument("--cpu-heads", type=int, default=8)
     ap.add_argument("--cpu-rows", type=int, default=4)
     args = ap.parse_args()

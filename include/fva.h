@@ -307,6 +307,40 @@ FVA_API int fva_rlb_plan(const double* head_load_ms, int n_heads, int n_ranks, d
                          double threshold, int max_per_rank, int32_t* rank_of_out, fva_rlb_move* moves_out,
                          int moves_capacity, int* n_moves_out);
 
+/*
+ * Slack-Aware Sparse Augmentation ([aixai] "Slack-Aware Sparse Augmentation (SASA)",
+ * "Sparse-routing frontend"; [PD] 方法揭秘), on a head split over n_ranks ranks.
+ *
+ * fva_sasa_budgets (host): blocks each rank may add. With L_crit the largest of
+ * rank_load_ms[0..n_ranks), a rank whose slack L_crit - L_r is >= n2 * L_crit gets
+ * floor(n1 * slack / block_ms) blocks, every other rank 0 (the pages' n1 = 0.8,
+ * n2 = 0.07; block_ms = compute time of one block). Returns FVA_OK or FVA_ERR_INVALID_ARG.
+ *
+ * fva_sasa_augment (device): adds to `mask` -- a mask fva_route produced for the same
+ * pooled Q/K, whose rows keep prefixes of their routing order -- each rank's budget of
+ * skipped (row, key block) entries with the largest routing importance P_ab (the row
+ * softmax of the block logits; ties to the lower head, query block, key block), over the
+ * rows of the heads with rank_of_head_dev[h] == r. A rank with fewer skipped entries than
+ * its budget gets all of them. The mask is rewritten in place: CSR, head_kept, tile lists
+ * and the work list in `order` (FVA_ORDER_*).
+ *   pooled_q_dev / pooled_k_dev: float64 [B, H, nB, d] as for fva_route;
+ *   rank_of_head_dev: int32 [B*H] device, values in [0, n_ranks) (others: FVA_DEVERR_BAD_LIST
+ *     in dev_status, and the head is left unchanged); n_ranks in [1, FVA_SASA_MAX_RANKS];
+ *   budget_dev: int64 [n_ranks] device (negative counts as 0);
+ *   added_dev: optional int64 [n_ranks] device, the entries added per rank;
+ *   workspace: fva_sasa_workspace_bytes(s) bytes, 16-byte aligned.
+ * Returns FVA_OK, FVA_ERR_INVALID_ARG, FVA_ERR_UNSUPPORTED_SHAPE, FVA_ERR_CAPACITY,
+ * FVA_ERR_WORKSPACE, FVA_ERR_ALIGNMENT or FVA_ERR_CUDA.
+ */
+#define FVA_SASA_MAX_RANKS 64
+FVA_API int fva_sasa_budgets(const double* rank_load_ms, int n_ranks, double block_ms, double n1, double n2,
+                             int64_t* budget_out);
+FVA_API size_t fva_sasa_workspace_bytes(const fva_shape* s);
+FVA_API int fva_sasa_augment(const fva_shape* s, const double* pooled_q_dev, const double* pooled_k_dev,
+                             const int32_t* rank_of_head_dev, int n_ranks, const int64_t* budget_dev, int order,
+                             const fva_mask* mask, void* workspace_dev, size_t workspace_bytes, int64_t* added_dev,
+                             int32_t* dev_status, fva_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

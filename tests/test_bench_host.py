@@ -34,9 +34,11 @@ def test_measured_sm_imbalance_balanced():
 def test_rlb_report_on_hand_costs():
     # 4 heads x 2 tiles; head loads in tile steps 18, 2, 2, 2 -> ranks (2 ranks) 20 | 4
     costs = np.array([9, 9, 1, 1, 1, 1, 1, 1], dtype=np.int64)
-    r = bench.rlb_report(costs, 4, 2, t_attn_ms=24.0, head_bytes=0.0, ranks=2)  # 1 ms per tile step
+    r, plan = bench.rlb_report(costs, 4, 2, t_attn_ms=24.0, head_bytes=0.0, ranks=2)  # 1 ms per tile step
     assert r["before"]["makespan_ms"] == pytest.approx(20.0)
     assert r["before"]["max_over_min"] == pytest.approx(5.0)
     # moving head 0 (18) would overshoot; head 1 (2) gives 18 | 6
     assert r["moves"] == [[1, 0, 1]]
     assert r["after"]["makespan_ms"] == pytest.approx(18.0)
+    np.testing.assert_array_equal(plan["rank_of"], [0, 1, 1, 1])
+    np.testing.assert_array_equal(plan["home"], [0, 0, 1, 1])
