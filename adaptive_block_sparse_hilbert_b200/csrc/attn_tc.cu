@@ -37,13 +37,6 @@ constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 64;   // keys per step (one key block)
 constexpr uint32_t kTmemCols = 256;
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
-// Every kPolyEvery-th pair of scores can take exp2 on the FMA pipe instead of MUFU (build
-// option; 0 = never). Measured on B200 at d = 128, moving 1/8 .. 1/2 of the exponentials
-// to the polynomial made the kernel slower: the softmax is issue/latency bound, not MUFU bound.
-#ifndef FVA_POLY_EVERY
-#define FVA_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = FVA_POLY_EVERY;
 
 // Bounded wait taken by a whole warp: the result is the same on every lane, so the
 // warp stays converged for the .sync.aligned TMEM instructions that follow.
@@ -350,10 +343,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           l_sum *= ex2_approx(m_ref - m_new);
           m_ref = m_new;
         }
-        // p = 2^(s * scale * log2 e - m_ref) on pairs of scores: one packed FFMA, then
-        // either two MUFU.EX2 or (every kPolyEvery-th pair) the FMA-pipe polynomial, which
-        // keeps the MUFU pipe from being the step's bottleneck; the row sum runs in two
-        // packed accumulators
+        // p = 2^(s * scale * log2 e - m_ref) on pairs of scores: one packed FFMA and two
+        // MUFU.EX2; the row sum runs in two packed accumulators
         const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
         const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
         uint64_t acc2[2] = {0ull, 0ull};
@@ -361,12 +352,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         for (int c = 0; c < 32; ++c) {
           const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])),
                                             sc2, nm2));
-          uint64_t p2;
-          if (kPolyEvery > 0 && (c % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
-            p2 = exp2_poly_pair(x.x, x.y);
-          } else {
-            p2 = f2_pack(ex2_approx(x.x), ex2_approx(x.y));
-          }
+          const uint64_t p2 = f2_pack(ex2_approx(x.x), ex2_approx(x.y));
           const float2 p = f2_unpack(p2);
           pk[c] = VF16 ? pack_f16x2(p.x, p.y) : pack_bf16x2(p.x, p.y);
           acc2[c & 1] = f2_add(acc2[c & 1], p2);

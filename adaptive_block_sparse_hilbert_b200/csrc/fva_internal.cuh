@@ -248,15 +248,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       FVA_W8(0), FVA_W8(8), FVA_W8(16), FVA_W8(24)
       : "memory");
 }
-// Store 16 consecutive 32-bit TMEM columns and wait.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-      FVA_W8(0), FVA_W8(8)
-      : "memory");
-}
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -275,17 +266,6 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t v;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(v) : "f"(hi), "f"(lo));
   return v;
-}
-// The two floats a packed pair holds again (exact widening).
-__device__ __forceinline__ float2 unpack_bf16x2(uint32_t v) {
-  return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
-}
-__device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
-  float lo, hi;
-  asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
-      : "=f"(lo), "=f"(hi)
-      : "r"(v));
-  return make_float2(lo, hi);
 }
 
 // ---- packed fp32 pairs (sm_100 f32x2 arithmetic) ------------------------------------------
@@ -315,29 +295,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x for a pair of floats on the FMA pipe (no MUFU): x = j + f with j = rint(x) and
-// f in [-1/2, 1/2]; 2^f by a degree-4 polynomial (coefficients fitted for this library
-// by weighted least squares in relative error on Chebyshev nodes; max relative error
-// 2.7e-6 in fp32 Horner form), then j is added to the exponent field. Inputs below -126
-// are clamped to -126 (result ~1e-38); inputs are at most 2^8 here.
-__device__ __forceinline__ uint64_t exp2_poly_pair(float x0, float x1) {
-  const float magic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
-  const uint64_t xc = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-  const uint64_t t = f2_add(xc, f2_pack(magic, magic));
-  const uint64_t j = f2_add(t, f2_pack(-magic, -magic));
-  const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), xc);
-  uint64_t p = f2_fma(f2_pack(0.009570096619427204f, 0.009570096619427204f), f,
-                      f2_pack(0.05591785907745361f, 0.05591785907745361f));
-  p = f2_fma(p, f, f2_pack(0.240247443318367f, 0.240247443318367f));
-  p = f2_fma(p, f, f2_pack(0.6931217908859253f, 0.6931217908859253f));
-  p = f2_fma(p, f, f2_pack(0.9999992847442627f, 0.9999992847442627f));
-  // bits(t) = bits(1.5 * 2^23) + j, and bits(1.5 * 2^23) << 23 == 0 modulo 2^32
-  const float2 tf = f2_unpack(t);
-  const float2 pf = f2_unpack(p);
-  const uint32_t lo = __float_as_uint(pf.x) + (__float_as_uint(tf.x) << 23);
-  const uint32_t hi = __float_as_uint(pf.y) + (__float_as_uint(tf.y) << 23);
-  return (static_cast<uint64_t>(hi) << 32) | lo;
-}
 
 // Warp reductions with a fixed butterfly order (deterministic).
 __device__ __forceinline__ double warp_sum_d(double v) {

@@ -497,6 +497,13 @@ def run_gpu(args):
     issued_flops = float(np.mean([4 * d * 128 * 64 * x[2].sum() for x in per_step]))
     dense_flops = float(4 * d * BH * N * N)
     reorder_bytes = float(6 * wl.B * N * wl.H * d * (2 if wl.dtype == "bf16" else 4) + 2 * BH * nB * d * 8)
+    # routing: pooled Q, K read (float64) + row_ptr, col_idx, head_kept, tile_ptr, tile_col,
+    # tile_cost and work list written; the logit GEMM is 2 d FLOP per (a, b) logit
+    n_tiles = BH * ((nB + 1) // 2)
+    union_entries = float(np.mean([x[2].sum() for x in per_step]))
+    route_bytes = float(2 * BH * nB * d * 8 + 4 * (BH * nB + 1) + 4 * kept + 8 * BH + 4 * (n_tiles + 1)
+                        + 4 * union_entries + 8 * n_tiles)
+    route_gemm_flop = float(2 * d * BH * nB * nB)
     drift = None
     if len(per_step) > 1:
         kept_heads = [x[3] for x in per_step]
@@ -612,6 +619,14 @@ def run_gpu(args):
             "dense_attn_tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 1) if dense_ms else None,
             "reorder_gbs": round(reorder_bytes / (t_reorder * 1e-3) / 1e9, 1),
             "reorder_hbm_frac": round(reorder_bytes / (t_reorder * 1e-3) / 1e9 / hbm, 4),
+            "route": {"gbs": round(route_bytes / (t_route * 1e-3) / 1e9, 1),
+                      "hbm_frac": round(route_bytes / (t_route * 1e-3) / 1e9 / hbm, 4),
+                      "bound": "fp64 ALU (block logits) + selection",
+                      "logit_gemm_fp64_tflops": round(route_gemm_flop / (t_route * 1e-3) / 1e12, 2),
+                      "note": "GB/s of algorithmic bytes over the whole routing stage; the fp64 rate is a lower "
+                              "bound for the GEMM alone (the stage time includes selection and emit)"},
+            "reorder_plus_route_hbm_frac": round((reorder_bytes + route_bytes) / ((t_reorder + t_route) * 1e-3) / 1e9
+                                                 / hbm, 4),
             "roofline": {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": round(achieved_tf / peak_tf, 4), "traffic": traffic,
                          "kernel": "attn_bf16_kernel (fva_sparse_attn)",
