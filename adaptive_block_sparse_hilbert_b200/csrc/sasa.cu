@@ -154,19 +154,35 @@ __global__ void __launch_bounds__(256) sasa_ties_count_kernel(const uint64_t* __
   if (lane == 0) tie_take[r] = n;
 }
 
-// rows in (head, query block) order take the ties each rank still needs
-__global__ void sasa_ties_alloc_kernel(int64_t rows, int nB, const int32_t* __restrict__ rank_of, int R,
-                                       const long long* __restrict__ need, int32_t* tie_take) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  long long left[64];
-  for (int r = 0; r < R; ++r) left[r] = need[r] > 0 ? need[r] : 0;
-  for (int64_t row = 0; row < rows; ++row) {
-    const int n = tie_take[row];
-    if (n == 0) continue;
-    const int rk = rank_of_row(rank_of, row, nB, R);
-    const long long t = rk < 0 ? 0 : (left[rk] < n ? left[rk] : n);
-    if (rk >= 0) left[rk] -= t;
-    tie_take[row] = static_cast<int32_t>(t);
+// rows in (head, query block) order take the ties each rank still needs. Ties are rare:
+// each thread flags whether its contiguous chunk of rows holds any, and one thread then
+// walks only the flagged chunks, in row order.
+__global__ void __launch_bounds__(1024) sasa_ties_alloc_kernel(int64_t rows, int nB,
+                                                               const int32_t* __restrict__ rank_of, int R,
+                                                               const long long* __restrict__ need, int32_t* tie_take) {
+  __shared__ int has[1024];
+  __shared__ long long left[kSasaMaxRanks];
+  const int64_t chunk = (rows + blockDim.x - 1) / blockDim.x;
+  const int64_t lo = threadIdx.x * chunk;
+  const int64_t hi = lo + chunk < rows ? lo + chunk : rows;
+  int any = 0;
+  for (int64_t row = lo; row < hi; ++row) any |= tie_take[row] != 0;
+  has[threadIdx.x] = any;
+  if (threadIdx.x < R) left[threadIdx.x] = need[threadIdx.x] > 0 ? need[threadIdx.x] : 0;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  for (int c = 0; c < static_cast<int>(blockDim.x); ++c) {
+    if (!has[c]) continue;
+    const int64_t clo = c * chunk;
+    const int64_t chi = clo + chunk < rows ? clo + chunk : rows;
+    for (int64_t row = clo; row < chi; ++row) {
+      const int n = tie_take[row];
+      if (n == 0) continue;
+      const int rk = rank_of_row(rank_of, row, nB, R);
+      const long long t = rk < 0 ? 0 : (left[rk] < n ? left[rk] : n);
+      if (rk >= 0) left[rk] -= t;
+      tie_take[row] = static_cast<int32_t>(t);
+    }
   }
 }
 
@@ -246,7 +262,7 @@ cudaError_t launch_sasa(const Dims& D, const double* pq, const double* pk, const
     sasa_pick_kernel<<<1, kSasaMaxRanks, 0, st>>>(hist, R, shift, prefix, pmask, need, dev_status);
   }
   sasa_ties_count_kernel<<<row_grid, 256, 0, st>>>(keys, D.rows, nB, rank_of, R, prefix, need, tie_take);
-  sasa_ties_alloc_kernel<<<1, 32, 0, st>>>(D.rows, nB, rank_of, R, need, tie_take);
+  sasa_ties_alloc_kernel<<<1, 1024, 0, st>>>(D.rows, nB, rank_of, R, need, tie_take);
   sasa_bits_kernel<<<row_grid, 256, 0, st>>>(keys, D.rows, nB, nWords, rank_of, R, prefix, pmask, need, tie_take,
                                               ws.bits, ws.row_cnt);
   e = cudaGetLastError();
