@@ -222,6 +222,15 @@ int fva_route(const fva_shape* s, const void* q_bhnd_dev, const void* k_bhnd_dev
   return cuda_status(launch_route(D, pq, pk, p, k_floor, order, mask, rs, dev_status, stream));
 }
 
+int fva_copy_strided(void* dst, size_t dst_pitch_bytes, const void* src, size_t src_pitch_bytes, size_t width_bytes,
+                     int64_t rows, fva_stream_t stream) {
+  if (!dst || !src || rows < 0) return FVA_ERR_INVALID_ARG;
+  if (width_bytes > dst_pitch_bytes || width_bytes > src_pitch_bytes) return FVA_ERR_INVALID_ARG;
+  if (rows == 0 || width_bytes == 0) return FVA_OK;
+  return cuda_status(cudaMemcpy2DAsync(dst, dst_pitch_bytes, src, src_pitch_bytes, width_bytes,
+                                       static_cast<size_t>(rows), cudaMemcpyDefault, stream));
+}
+
 size_t fva_sasa_workspace_bytes(const fva_shape* s) {
   Dims D;
   if (!make_dims(s, &D)) return 0;

@@ -93,6 +93,7 @@ def _load():
         "fva_tiles_workspace_bytes": (sz, [S]),
         "fva_hilbert_perm": (i32, [S, P, P, P]),
         "fva_curve_perm": (i32, [S, i32, P, P, P, P]),
+        "fva_copy_strided": (i32, [P, sz, P, sz, sz, i64, P]),
         "fva_sasa_budgets": (i32, [ctypes.POINTER(ctypes.c_double), i32, dbl, dbl, dbl, ctypes.POINTER(ctypes.c_int64)]),
         "fva_sasa_workspace_bytes": (sz, [S]),
         "fva_sasa_augment": (i32, [S, P, P, P, i32, P, i32, M, P, sz, P, P, P]),
@@ -117,7 +118,7 @@ EXPORTED = (
     "fva_tile_capacity", "fva_route_workspace_bytes", "fva_tiles_workspace_bytes", "fva_hilbert_perm", "fva_reorder",
     "fva_pool", "fva_route", "fva_build_tiles", "fva_sparse_attn", "fva_dense_attn", "fva_route_noalloc",
     "fva_set_cta_trace", "fva_rlb_plan", "fva_curve_perm", "fva_sasa_budgets", "fva_sasa_workspace_bytes",
-    "fva_sasa_augment",
+    "fva_sasa_augment", "fva_copy_strided",
 )
 
 
@@ -296,6 +297,12 @@ def fva_route_noalloc(s, q, k, pooled_q, pooled_k, p, k_floor, mask: Mask, order
     _check("fva_route_noalloc", _lib.fva_route_noalloc(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(pooled_q),
                                                        _ptr(pooled_k), float(p), int(k_floor), int(order),
                                                        ctypes.byref(m), _ptr(dev_status), _stream(stream)))
+
+
+def fva_copy_strided(dst, dst_pitch_bytes, src, src_pitch_bytes, width_bytes, rows, stream=None):
+    """Pitched async copy between device and page-locked host memory (pointers or tensors)."""
+    _check("fva_copy_strided", _lib.fva_copy_strided(_ptr(dst), int(dst_pitch_bytes), _ptr(src), int(src_pitch_bytes),
+                                                     int(width_bytes), int(rows), _stream(stream)))
 
 
 def fva_sasa_workspace_bytes(s): return _lib.fva_sasa_workspace_bytes(ctypes.byref(s))

@@ -65,3 +65,76 @@ class SparseAttentionLayer:
         self.attend(stream)
         self.restore_output(o_out, stream)
         return o_out
+
+
+class HostPipelinedLayer:
+    """One layer from page-locked host Q, K, V [B, N, H, d] to host O, pipelined over head
+    groups: one stream copies group g+1's head slices in while another runs group g's
+    reorder -> route -> attention -> inverse reorder and a third copies group g-1's output
+    back. Heads are independent along the whole path, so every group is an ordinary
+    SparseAttentionLayer on a shape with fewer heads, and the output equals the one-shot
+    layer's bit for bit.
+
+        layer = HostPipelinedLayer(shape, p=0.9, k_floor=4, groups=8)
+        layer.forward(q_host, k_host, v_host, o_host)   # pinned CPU tensors, raster order
+    """
+
+    def __init__(self, shape: fva.fva_shape, p: float, k_floor: int, groups: int = 8,
+                 order: int = fva.FVA_ORDER_HEAD_LPT, device: str = "cuda", v_fp16: bool = True,
+                 curve: int = fva.FVA_CURVE_HILBERT):
+        s = shape
+        H = s.H
+        groups = max(1, min(int(groups), H))
+        sizes = [H // groups + (1 if g < H % groups else 0) for g in range(groups)]
+        self.shape = s
+        self.heads = []  # (first head, count) per group
+        h0 = 0
+        for n in sizes:
+            self.heads.append((h0, n))
+            h0 += n
+        self.N = fva.fva_num_tokens(s)
+        dt = torch.bfloat16 if s.dtype == fva.FVA_BF16 else torch.float32
+        self.esize = 2 if s.dtype == fva.FVA_BF16 else 4
+        self.layers, self.q_in, self.k_in, self.v_in, self.o_out = [], [], [], [], []
+        for _, n in self.heads:
+            gs = fva.make_shape(s.B, n, s.d, s.T, s.Hg, s.Wg, s.dtype)
+            self.layers.append(SparseAttentionLayer(gs, p, k_floor, order, device, v_fp16, curve))
+            for lst in (self.q_in, self.k_in, self.v_in, self.o_out):
+                lst.append(torch.empty((s.B, self.N, n, s.d), dtype=dt, device=device))
+        self.s_in = torch.cuda.Stream(device=device)
+        self.s_comp = torch.cuda.Stream(device=device)
+        self.s_out = torch.cuda.Stream(device=device)
+
+    def forward(self, q_host, k_host, v_host, o_host):
+        """Enqueue the layer; returns the stream whose completion means o_host is written
+        (the caller's current stream is made to wait on it)."""
+        s = self.shape
+        row = s.H * s.d * self.esize
+        rows = s.B * self.N
+        cur = torch.cuda.current_stream()
+        self.s_in.wait_stream(cur)
+        self.s_comp.wait_stream(cur)
+        self.s_out.wait_stream(cur)
+        ready = []
+        for (h0, n), qd, kd, vd in zip(self.heads, self.q_in, self.k_in, self.v_in):
+            width = n * s.d * self.esize
+            for dst, src in ((qd, q_host), (kd, k_host), (vd, v_host)):
+                fva.fva_copy_strided(dst, width, src[:, :, h0:h0 + n, :], row, width, rows, self.s_in)
+            ev = torch.cuda.Event()
+            ev.record(self.s_in)
+            ready.append(ev)
+        for g, ((h0, n), layer) in enumerate(zip(self.heads, self.layers)):
+            self.s_comp.wait_event(ready[g])
+            layer.forward(self.q_in[g], self.k_in[g], self.v_in[g], self.o_out[g], self.s_comp)
+            done = torch.cuda.Event()
+            done.record(self.s_comp)
+            self.s_out.wait_event(done)
+            width = n * s.d * self.esize
+            fva.fva_copy_strided(o_host[:, :, h0:h0 + n, :], row, self.o_out[g], width, width, rows, self.s_out)
+        cur.wait_stream(self.s_out)
+        cur.wait_stream(self.s_comp)
+        return self.s_out
+
+    def dev_status(self):
+        """Largest device error code any group reported (0 = none)."""
+        return max(int(l.dev_status.item()) for l in self.layers)

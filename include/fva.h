@@ -341,6 +341,18 @@ FVA_API int fva_sasa_augment(const fva_shape* s, const double* pooled_q_dev, con
                              const fva_mask* mask, void* workspace_dev, size_t workspace_bytes, int64_t* added_dev,
                              int32_t* dev_status, fva_stream_t stream);
 
+/*
+ * Strided asynchronous copy (data movement for the host-pipelined layer; the pages have
+ * no counterpart): `rows` rows of `width_bytes` each, from src (consecutive rows
+ * src_pitch_bytes apart) to dst (dst_pitch_bytes apart), enqueued on `stream`. Either
+ * pointer may be device memory or page-locked host memory (the direction follows from the
+ * pointers). With host rows of H * d elements and a device buffer of G * d, this moves the
+ * slice of G heads of a [B, N, H, d] tensor in one call. Returns FVA_OK,
+ * FVA_ERR_INVALID_ARG (null pointer, width > a pitch, negative sizes) or FVA_ERR_CUDA.
+ */
+FVA_API int fva_copy_strided(void* dst, size_t dst_pitch_bytes, const void* src, size_t src_pitch_bytes,
+                             size_t width_bytes, int64_t rows, fva_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -132,3 +132,12 @@ def test_curve_perm_rejects_unknown_curve():
     s = fva.make_shape(1, 1, 64, 2, 8, 8, "bf16")
     assert fva.lib().fva_curve_perm(ctypes.byref(s), 7, 1024, 2048, None, None) == fva.FVA_ERR_INVALID_ARG
     assert fva.lib().fva_curve_perm(ctypes.byref(s), fva.FVA_CURVE_RECT, None, 2048, None, None) == fva.FVA_ERR_INVALID_ARG
+
+
+def test_copy_strided_argument_checks():
+    L = fva.lib()
+    assert L.fva_copy_strided(None, 16, 1024, 16, 16, 1, None) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_copy_strided(1024, 8, 2048, 16, 16, 1, None) == fva.FVA_ERR_INVALID_ARG   # width > dst pitch
+    assert L.fva_copy_strided(1024, 16, 2048, 8, 16, 1, None) == fva.FVA_ERR_INVALID_ARG   # width > src pitch
+    assert L.fva_copy_strided(1024, 16, 2048, 16, 16, -1, None) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_copy_strided(1024, 16, 2048, 16, 16, 0, None) == fva.FVA_OK               # nothing to move
