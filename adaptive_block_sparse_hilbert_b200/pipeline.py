@@ -67,6 +67,27 @@ class SparseAttentionLayer:
         return o_out
 
 
+def ramp_sizes(H: int, steady: int = 4):
+    """Head-group sizes for the pipelined layer: groups of 1, 2, 3 heads first (the first
+    group's copy-in is the only one nothing overlaps), then `steady`-head groups, and a
+    half-size last group (its copy-out is the only one after the compute). Sums to H."""
+    sizes, left = [], H
+    for n in (1, 2, 3):
+        n = min(n, steady, left)
+        if n > 0:
+            sizes.append(n)
+            left -= n
+    tail = min(max(1, steady // 2), left)
+    left -= tail
+    while left > 0:
+        n = min(steady, left)
+        sizes.append(n)
+        left -= n
+    if tail > 0:
+        sizes.append(tail)
+    return sizes
+
+
 class HostPipelinedLayer:
     """One layer from page-locked host Q, K, V [B, N, H, d] to host O, pipelined over head
     groups: one stream copies group g+1's head slices in while another runs group g's
@@ -75,17 +96,25 @@ class HostPipelinedLayer:
     SparseAttentionLayer on a shape with fewer heads, and the output equals the one-shot
     layer's bit for bit.
 
-        layer = HostPipelinedLayer(shape, p=0.9, k_floor=4, groups=8)
+        layer = HostPipelinedLayer(shape, p=0.9, k_floor=4)   # ramp of head groups
         layer.forward(q_host, k_host, v_host, o_host)   # pinned CPU tensors, raster order
     """
 
-    def __init__(self, shape: fva.fva_shape, p: float, k_floor: int, groups: int = 8,
+    def __init__(self, shape: fva.fva_shape, p: float, k_floor: int, groups=None,
                  order: int = fva.FVA_ORDER_HEAD_LPT, device: str = "cuda", v_fp16: bool = True,
-                 curve: int = fva.FVA_CURVE_HILBERT):
+                 curve: int = fva.FVA_CURVE_HILBERT, sizes=None):
+        """groups: None for the ramp schedule (ramp_sizes), or a number of equal groups;
+        sizes: explicit head counts per group (overrides groups)."""
         s = shape
         H = s.H
-        groups = max(1, min(int(groups), H))
-        sizes = [H // groups + (1 if g < H % groups else 0) for g in range(groups)]
+        if sizes is None and groups is None:
+            sizes = ramp_sizes(H)
+        elif sizes is None:
+            groups = max(1, min(int(groups), H))
+            sizes = [H // groups + (1 if g < H % groups else 0) for g in range(groups)]
+        sizes = [int(n) for n in sizes if int(n) > 0]
+        if sum(sizes) != H:
+            raise ValueError(f"group sizes {sizes} do not add up to {H} heads")
         self.shape = s
         self.heads = []  # (first head, count) per group
         h0 = 0

@@ -574,6 +574,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     e2e_serial_ms = e0.elapsed_time(e1) / n_e2e
     piped = pipeline.HostPipelinedLayer(s, wl.p, wl.k_floor, groups=args.e2e_groups, device=dev, curve=curve)
+    e2e_sizes = [n for _, n in piped.heads]
     for _ in range(2):
         piped.forward(hq, hk, hv, ho)
     torch.cuda.synchronize()
@@ -652,7 +653,7 @@ def run_gpu(args):
             "e2e": {"value": round(whole_job_ms_per_layer(e2e_ms, world), 3), "unit": "ms/layer",
                     "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h),
-                    "how": f"pipelined over {args.e2e_groups} head groups (copy in / compute / copy out "
+                    "how": f"pipelined over head groups of {e2e_sizes} heads (copy in / compute / copy out "
                            f"on three streams)", "serial_ms": round(whole_job_ms_per_layer(e2e_serial_ms, world), 3)},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clk,
@@ -683,7 +684,8 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sasa", action="store_true", help="skip the slack-aware augmentation report")
-    ap.add_argument("--e2e-groups", type=int, default=8, help="head groups of the host-pipelined end-to-end run")
+    ap.add_argument("--e2e-groups", type=int, default=None,
+                    help="equal head groups of the host-pipelined end-to-end run (default: a ramp 1, 2, 3, 4, ..., 2)")
     ap.add_argument("--cpu-heads", type=int, default=8)
     ap.add_argument("--cpu-rows", type=int, default=4)
     args = ap.parse_args()

@@ -42,3 +42,13 @@ def test_rlb_report_on_hand_costs():
     assert r["after"]["makespan_ms"] == pytest.approx(18.0)
     np.testing.assert_array_equal(plan["rank_of"], [0, 1, 1, 1])
     np.testing.assert_array_equal(plan["home"], [0, 0, 1, 1])
+
+
+@pytest.mark.parametrize("H", [1, 2, 3, 5, 6, 7, 10, 40, 48, 129])
+def test_ramp_sizes(H):
+    from adaptive_block_sparse_hilbert_b200 import pipeline
+    sizes = pipeline.ramp_sizes(H)
+    assert sum(sizes) == H and min(sizes) >= 1 and max(sizes) <= 4
+    assert sizes[: 3] == [1, 2, 3][: len(sizes[:3])] or H < 6
+    if H >= 10:
+        assert sizes[:3] == [1, 2, 3] and sizes[-1] == 2

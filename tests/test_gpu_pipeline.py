@@ -9,7 +9,7 @@ from tests import _common as C
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("H,groups", [(5, 3), (4, 4), (6, 1)])
+@pytest.mark.parametrize("H,groups", [(5, 3), (4, 4), (6, 1), (7, None)])
 def test_pipelined_equals_one_shot(H, groups):
     import torch
     from adaptive_block_sparse_hilbert_b200 import fva, pipeline
