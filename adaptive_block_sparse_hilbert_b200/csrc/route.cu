@@ -123,10 +123,12 @@ constexpr int kNBK = 128;                       // buckets per refinement level
 constexpr int kMaxLevels = 12;
 constexpr double kFix = 4503599627370496.0;     // 2^52: fixed-point unit of importance
 
+// Shared memory of one row's warp. The importances exp(s - max) are recomputed where they
+// are needed rather than kept (the same operation on the same inputs, so the same bits):
+// an fp64 copy of them would double the arena and halve the warps that fit on an SM.
 struct WarpArena {
   double* s;          // [nB] the row's logits
-  double* e;          // [nB] exp(s - max)
-  uint64_t* hw;       // [kNBK] bucket mass (fixed point)
+  uint64_t* hw;       // [kNBK] bucket mass (fixed point); last: masses of the final candidates
   int32_t* list;      // [nB] candidate block indices
   int32_t* hcnt;      // [kNBK] bucket counts
   uint32_t* words;    // [nWords] kept bitmask of the row
@@ -134,7 +136,6 @@ struct WarpArena {
 
 __host__ __device__ inline size_t warp_arena_bytes(int nB, int nWords) {
   size_t b = 0;
-  b += align_up(static_cast<size_t>(nB) * 8, 16);
   b += align_up(static_cast<size_t>(nB) * 8, 16);
   b += kNBK * 8;
   b += align_up(static_cast<size_t>(nB) * 4, 16);
@@ -147,8 +148,6 @@ __device__ inline WarpArena make_arena(uint8_t* base, int nB, int nWords) {
   WarpArena A;
   size_t off = 0;
   A.s = reinterpret_cast<double*>(base + off);
-  off += align_up(static_cast<size_t>(nB) * 8, 16);
-  A.e = reinterpret_cast<double*>(base + off);
   off += align_up(static_cast<size_t>(nB) * 8, 16);
   A.hw = reinterpret_cast<uint64_t*>(base + off);
   off += kNBK * 8;
@@ -205,7 +204,7 @@ __device__ Pivot select_pivot(const WarpArena& A, int nB, double smax, double sm
       bk = bk < 0 ? 0 : (bk >= kNBK ? kNBK - 1 : bk);
       atomicAdd(&A.hcnt[bk], 1);
       if (by_mass) atomicAdd(reinterpret_cast<unsigned long long*>(&A.hw[bk]),
-                             static_cast<unsigned long long>(fixed_mass(A.e[b], zscale)));
+                             static_cast<unsigned long long>(fixed_mass(exp(s - smax), zscale)));
     }
     __syncwarp();
     // lane owns buckets 4*lane .. 4*lane+3
@@ -302,6 +301,13 @@ __device__ Pivot select_pivot(const WarpArena& A, int nB, double smax, double sm
     for (int i = lane; i < c; i += 32) A.list[i] = i;
     __syncwarp();
   }
+  // masses of the remaining candidates, kept in the bucket array when they fit (the
+  // levels normally leave <= 32; equal logits can leave more, which recompute)
+  const bool cached = by_mass && c <= kNBK;
+  if (cached) {
+    for (int i = lane; i < c; i += 32) A.hw[i] = fixed_mass(exp(srow[A.list[i]] - smax), zscale);
+    __syncwarp();
+  }
   // exact order inside the remaining candidates: rank and inclusive cumulative mass
   int best_rank = 0x7fffffff;
   int best_b = -1;
@@ -318,12 +324,12 @@ __device__ Pivot select_pivot(const WarpArena& A, int nB, double smax, double sm
         const double sj = srow[bj];
         if (precedes(sj, bj, si, bi)) {
           ++rank;
-          if (by_mass) cw += fixed_mass(A.e[bj], zscale);
+          if (by_mass) cw += cached ? A.hw[j] : fixed_mass(exp(sj - smax), zscale);
         }
       }
       bool ok;
       if (by_mass) {
-        cw += fixed_mass(A.e[bi], zscale);
+        cw += cached ? A.hw[i] : fixed_mass(exp(si - smax), zscale);
         ok = static_cast<double>(above_w + cw) >= pth;
       } else {
         ok = (above_c + rank + 1 == cnt_target);
@@ -385,9 +391,7 @@ __global__ void route_select_kernel(const double* __restrict__ S, int nB, int nW
     smin = warp_min_d(smin);
     double z = 0.0;
     for (int b = lane; b < nB; b += 32) {
-      const double e = exp(srow[b] - smax);
-      A.e[b] = e;
-      z += e;
+      z += exp(srow[b] - smax);
     }
     const double Z = warp_sum_d(z);
     const double zscale = kFix / Z;
@@ -646,12 +650,24 @@ __global__ void __launch_bounds__(256) tile_cost_kernel(const uint32_t* __restri
 // ---------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------
+// Rows (warps) per CTA: the even count that fits the most warps on an SM (228 KB of shared
+// memory, 1 KB of it reserved per CTA, at most 64 warps), fewer rows per CTA on a tie; 0 if
+// not even two rows fit in one CTA's 227 KB.
 static int select_rows_per_cta(const Dims& D) {
   const size_t arena = warp_arena_bytes(static_cast<int>(D.nB), static_cast<int>(D.nWords));
-  constexpr size_t kBudget = 224 * 1024;  // dynamic shared memory per CTA (227 KB maximum)
-  int r = 8;
-  while (r > 2 && arena * r > kBudget) r -= 2;
-  return (arena * r > kBudget) ? 0 : r;
+  constexpr size_t kCta = 227 * 1024, kSm = 228 * 1024, kReserved = 1024;
+  int best = 0, best_warps = 0;
+  for (int r = 2; r <= 16; r += 2) {
+    const size_t smem = arena * r;
+    if (smem > kCta) break;
+    int ctas = static_cast<int>(kSm / (smem + kReserved));
+    if (ctas * r > 64) ctas = 64 / r;
+    if (ctas * r > best_warps) {
+      best_warps = ctas * r;
+      best = r;
+    }
+  }
+  return best;
 }
 
 static cudaError_t launch_order_and_emit(const Dims& D, const fva_mask* m, int order, const RouteScratch& ws,
