@@ -307,12 +307,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           for (int c = 0; c < 64; ++c)
             if (c >= nvalid) r[c] = 0xFF800000u;
         }
-        // row maximum of the raw scores: three-input max in four independent chains
+        // row maximum of the raw scores: four independent chains, seeded with r[0..7], then
+        // three-input maxima over r[8..63]
         float mx4[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) mx4[q] = __uint_as_float(r[q]);
+        for (int q = 0; q < 4; ++q) mx4[q] = fmaxf(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
 #pragma unroll
-        for (int c = 4; c < 64; c += 8) {
+        for (int c = 8; c < 64; c += 8) {
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             mx4[q] = fmax3(mx4[q], __uint_as_float(r[c + 2 * q]), __uint_as_float(r[c + 2 * q + 1]));
