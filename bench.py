@@ -469,6 +469,7 @@ def run_gpu(args):
 
     stage = np.array([[m[j].elapsed_time(m[j + 1]) for j in range(4)] for m in marks])
     t_reorder, t_route, t_attn, t_inv = [float(np.mean(stage[:, j])) for j in range(4)]
+    stage_median = [float(np.median(stage[:, j])) for j in range(4)]
     ms_step = total_ms / args.steps
 
     # mask statistics and algorithmic work (averaged over the drift steps, which the timed
@@ -630,6 +631,9 @@ def run_gpu(args):
             "density": round(kept / (BH * nB * nB), 4),
             "stage_ms": {"reorder_qkv": round(t_reorder, 4), "route": round(t_route, 4), "attn": round(t_attn, 4),
                          "inverse_o": round(t_inv, 4)},
+            "stage_ms_median": dict(zip(("reorder_qkv", "route", "attn", "inverse_o"),
+                                        (round(x, 4) for x in stage_median))),
+            "density_per_head": [round(float(x) / (nB * nB), 4) for x in per_step[0][3]],
             "dense_attn_ms": round(dense_ms, 3) if dense_ms else None,
             "dense_attn_tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 1) if dense_ms else None,
             "reorder_gbs": round(reorder_bytes / (t_reorder * 1e-3) / 1e9, 1),
