@@ -50,7 +50,7 @@ typedef struct CUstream_st* fva_stream_t; /* identical to cudaStream_t */
 enum {
   FVA_OK = 0,
   FVA_ERR_INVALID_ARG = -1,       /* null pointer, bad enum, p or k_floor out of range */
-  FVA_ERR_UNSUPPORTED_SHAPE = -2, /* shape/dtype combination this build does not handle */
+  FVA_ERR_UNSUPPORTED_SHAPE = -2, /* shape/dtype combination the library does not handle */
   FVA_ERR_CAPACITY = -3,          /* mask buffers smaller than fva_mask_capacity() etc. */
   FVA_ERR_CUDA = -4,              /* a CUDA runtime/driver call failed */
   FVA_ERR_DEVICE_TIMEOUT = -5,    /* reported through dev_status only */

@@ -17,7 +17,7 @@ Sources (the five pages about FVAttn, arXiv 2607.16190), cited by page and secti
 * [abs]    "FVAttn: Adaptive Sparse Attention with Runtime Load Balancing for Video
   Generation" (mlsanity.com) -- arXiv abstract.
 
-Readings taken where the pages leave a step open (each is listed in the design doc):
+Readings taken where the pages leave a step open:
 
 * Hilbert order: per frame, the 2-D curve over (y, x) on the enclosing 2^m square,
   out-of-grid cells skipped, frames concatenated in t order.

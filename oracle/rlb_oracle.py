@@ -19,7 +19,7 @@ Sources, cited by page and section:
   below a threshold or the migration budget is used up; the imbalance factor is the
   slowest rank's compute time over the fastest rank's.
 
-Readings where the pages leave a step open (listed in the design doc):
+Readings where the pages leave a step open:
 
 * Heads start in the contiguous Ulysses split: rank r owns heads [r H / R, (r+1) H / R).
 * The imbalance factor that stops the planner is max/min (the [PD] definition); the stop

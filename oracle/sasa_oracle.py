@@ -17,7 +17,7 @@ Sources, cited by page and section:
   idle-time budget and, from the blocks the sparse mask skipped, picks some in order of
   importance, keeping the extra compute within that budget.
 
-Readings where the pages leave a step open (listed in the design doc):
+Readings where the pages leave a step open:
 
 * The mode is chosen on the imbalance (slowest / fastest rank load) of the starting
   placement; below k1 nothing is added.

@@ -9,7 +9,7 @@ import numpy as np
 from adaptive_block_sparse_hilbert_b200 import synth
 import oracle as O
 
-# tolerances (bf16 inputs / fp32 inputs), see DESIGN.md "Acceptance"
+# acceptance tolerances for attention outputs (bf16 inputs / fp32 inputs)
 BF16_MAX_ABS = 2e-2
 BF16_MEAN_ABS = 2e-3
 F32_MAX_ABS = 1e-4
