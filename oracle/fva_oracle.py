@@ -27,7 +27,8 @@ Readings taken where the pages leave a step open:
 * Top-p cut: the minimal prefix whose cumulative importance is >= p; p >= 1 keeps all.
 * Top-k floor: the first min(k_floor, nB) blocks of the same order; the kept set is the
   union, i.e. the longer of the two prefixes.
-* Attention: softmax over the valid keys of the kept blocks only, no causal mask.
+* Attention: softmax over the valid keys of the kept blocks only, no causal mask. A row
+  that keeps no block (only a caller-made mask can have one) outputs zeros.
 
 Parity pins: every function here is pinned in tests/test_oracle_*.py against
 something other than itself (an independent L-system construction of the Hilbert
@@ -373,8 +374,13 @@ def lpt_order(cost: np.ndarray) -> np.ndarray:
 
 def attention_rows(q_nd: np.ndarray, k_nd: np.ndarray, v_nd: np.ndarray, keys: np.ndarray,
                    scale: float) -> np.ndarray:
-    """softmax(q k^T * scale) v over the given key rows, float64."""
+    """softmax(q k^T * scale) v over the given key rows, float64.
+
+    An empty key set (a caller-made mask row that keeps no block; routing always keeps
+    at least one) has no softmax; its output is taken to be zero."""
     q = np.asarray(q_nd, np.float64)
+    if len(keys) == 0:
+        return np.zeros((q.shape[0], np.asarray(v_nd).shape[-1]), dtype=np.float64)
     k = np.asarray(k_nd, np.float64)[keys]
     v = np.asarray(v_nd, np.float64)[keys]
     s = (q @ k.T) * scale

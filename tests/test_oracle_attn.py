@@ -49,6 +49,29 @@ def test_sparse_matches_masked_sdpa(p, kf):
     assert np.abs(got - O.dense_attention(q, k, v)).max() > 1e-3
 
 
+def test_empty_rows_give_zeros_and_leave_other_rows_alone():
+    # a caller-made mask: rows 0 and 3 keep nothing, the others keep scattered blocks
+    B, H, N, d = 1, 1, 64 * 5 + 11, 16
+    q, k, v = _rand((B, H, N, d), 21, 2.0), _rand((B, H, N, d), 22, 2.0), _rand((B, H, N, d), 23)
+    lists = [[], [0, 4], [2], [], [1, 3, 5], [5]]
+    nB = O.n_blocks(N)
+    assert nB == len(lists)
+    row_ptr = np.concatenate([[0], np.cumsum([len(x) for x in lists])]).astype(np.int64)
+    col_idx = np.array([b for x in lists for b in x], dtype=np.int64)
+    got = O.assemble(O.block_sparse_attention(q, k, v, row_ptr, col_idx), B, H, N, d)
+    mask = np.full((B, H, N, N), -np.inf)
+    for a, keep in enumerate(lists):
+        for b in keep:
+            mask[0, 0, a * 64:(a + 1) * 64, b * 64:(b + 1) * 64] = 0.0
+    want = _sdpa(q, k, v, mask)
+    for a, keep in enumerate(lists):
+        lo, hi = a * 64, min(a * 64 + 64, N)
+        if keep:
+            np.testing.assert_allclose(got[0, 0, lo:hi], want[0, 0, lo:hi], rtol=1e-12, atol=1e-12)
+        else:
+            assert np.all(got[0, 0, lo:hi] == 0.0)
+
+
 def test_p_one_equals_dense():
     B, H, N, d = 1, 1, 64 * 4 + 3, 16
     q, k, v = _rand((B, H, N, d), 7, 2.0), _rand((B, H, N, d), 8, 2.0), _rand((B, H, N, d), 9)
