@@ -127,7 +127,7 @@ int64_t fva_tile_capacity(const fva_shape* s) {
 
 size_t fva_route_workspace_bytes(const fva_shape* s, int need_pool) {
   Dims D;
-  if (!make_dims(s, &D)) return 0;
+  if (!make_dims(s, &D) || !route_shape_supported(D)) return 0;
   return route_scratch_layout(D, need_pool, nullptr, nullptr, nullptr, nullptr, true);
 }
 
@@ -233,7 +233,7 @@ int fva_copy_strided(void* dst, size_t dst_pitch_bytes, const void* src, size_t 
 
 size_t fva_sasa_workspace_bytes(const fva_shape* s) {
   Dims D;
-  if (!make_dims(s, &D)) return 0;
+  if (!make_dims(s, &D) || !route_shape_supported(D)) return 0;
   return route_scratch_layout(D, 0, nullptr, nullptr, nullptr, nullptr, true) + sasa_extra_bytes(D);
 }
 

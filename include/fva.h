@@ -79,7 +79,17 @@ enum {
   FVA_ORDER_HEAD_LPT = 2    /* heads by total cost desc (id asc), longest first inside a head */
 };
 
-/* Problem shape. block must be 64. dtype is FVA_F32 or FVA_BF16. */
+/* Problem shape. block must be 64. dtype is FVA_F32 or FVA_BF16.
+ * Limits (a shape outside them gives FVA_ERR_UNSUPPORTED_SHAPE, or -1 / 0 from the size
+ * queries, before anything is enqueued):
+ *   B, H, d, T, Hg, Wg >= 1 (an empty layer is rejected, not treated as a no-op);
+ *   Hg, Wg <= 65536; N = T*Hg*Wg <= 2^31 - 1; nB <= 524280; B*H <= 65535;
+ *   B*H*nB <= 2^31 - 1;
+ *   d * sizeof(dtype) in {64, 128, 256, 512, 1024} bytes;
+ *   routing (fva_route, fva_route_noalloc, fva_sasa_augment): nB <= 9458, the largest
+ *   count for which two rows' float64 working sets fit one CTA's 227 KB of shared
+ *   memory, and B*H*nB*nB <= 2^31 - 1 (int32 CSR offsets);
+ *   attention: see fva_sparse_attn. */
 typedef struct fva_shape {
   int32_t B, H, d;
   int32_t T, Hg, Wg;
@@ -145,7 +155,8 @@ FVA_API int64_t fva_num_tiles(const fva_shape* s);
 /* Entries col_idx / tile_col must hold: B*H*nB*nB and B*H*nPairs*nB. */
 FVA_API int64_t fva_mask_capacity(const fva_shape* s);
 FVA_API int64_t fva_tile_capacity(const fva_shape* s);
-/* Bytes of workspace fva_route needs (with need_pool != 0: also room to pool Q and K). */
+/* Bytes of workspace fva_route needs (with need_pool != 0: also room to pool Q and K);
+ * 0 when the shape is outside the routing limits above. */
 FVA_API size_t fva_route_workspace_bytes(const fva_shape* s, int need_pool);
 
 /*
@@ -242,6 +253,8 @@ FVA_API int fva_build_tiles(const fva_shape* s, const fva_mask* mask, int order,
  *   s->dtype == FVA_F32 (CUDA cores, d in {32, 64, 128}): v_dtype must be FVA_F32.
  * scale <= 0 selects 1/sqrt(d). Reads mask->tile_ptr, tile_col, worklist (bf16) or
  * mask->row_ptr, col_idx (fp32). o must not overlap q, k or v.
+ * A row that keeps no key block (possible only in a caller-made mask: fva_route keeps at
+ * least one block per row) has an empty softmax; its output rows are written as zeros.
  */
 FVA_API int fva_sparse_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev,
                             int v_dtype, const fva_mask* mask, void* o_dev, float scale, int32_t* dev_status,

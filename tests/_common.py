@@ -165,3 +165,10 @@ def sample_rows(row_ptr, BH, nB, n_per_head, seed):
 
 def default_scale(d):
     return 1.0 / math.sqrt(d)
+
+
+def largest_routable_workload():
+    """One head at the routing kernel's largest block count: 778 x 778 = 605,284 tokens,
+    nB = 9458 (a ragged tail of 36), d = 64. Heads drawn with tau in logU(2, 2.5) give a
+    density near 0.18 with row lengths from a few dozen to thousands of blocks."""
+    return synth.custom_workload(1, 778, 778, 1, 64, "bf16", seed=41, tau=("logU", 2.0, 2.5))

@@ -68,6 +68,29 @@ def test_invalid_shapes_rejected():
         assert fva.fva_route_workspace_bytes(s) == 0
 
 
+def test_routing_limit_on_block_count():
+    """Routing keeps two rows' float64 working sets in one CTA's shared memory, which
+    bounds nB at 9458; one block more is rejected on the host before any launch."""
+    P = ctypes.c_void_p
+    one = P(16)  # non-null dummy pointer; every call below fails validation first
+    ok = fva.make_shape(1, 1, 64, 1, 778, 778)        # N = 605,284: nB = 9458
+    over = fva.make_shape(1, 1, 64, 10, 1, 60532)     # N = 605,320: nB = 9459
+    assert fva.fva_num_blocks(ok) == 9458 and fva.fva_num_blocks(over) == 9459
+    assert fva.fva_route_workspace_bytes(ok, 0) > 0 and fva.fva_route_workspace_bytes(ok, 1) > 0
+    assert fva.fva_sasa_workspace_bytes(ok) > 0
+    assert fva.fva_route_workspace_bytes(over, 0) == 0 and fva.fva_route_workspace_bytes(over, 1) == 0
+    assert fva.fva_sasa_workspace_bytes(over) == 0
+    small = fva.fva_mask(16, 16, 10, 16, 16, 16, 10, 16, 16)
+    args = (one, one, None, None, 0.9, 4, 2, ctypes.byref(small), one, 1 << 30, None, None)
+    assert fva.call_raw("fva_route", ctypes.byref(over), *args) == fva.FVA_ERR_UNSUPPORTED_SHAPE
+    # the limit shape passes the shape checks and stops at the (too small) mask capacity
+    assert fva.call_raw("fva_route", ctypes.byref(ok), *args) == fva.FVA_ERR_CAPACITY
+    assert fva.call_raw("fva_route_noalloc", ctypes.byref(over), one, one, None, None, 0.9, 4, 2,
+                        ctypes.byref(small), None, None) == fva.FVA_ERR_UNSUPPORTED_SHAPE
+    # tile building from a caller-made mask has no such limit
+    assert fva.fva_tiles_workspace_bytes(over) > 0
+
+
 def test_host_validation_before_any_launch():
     s = fva.make_shape(1, 2, 64, 4, 16, 16, "f32")
     P = ctypes.c_void_p

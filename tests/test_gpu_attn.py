@@ -149,11 +149,22 @@ def test_disjoint_pair_lists_and_all_blocks(d):
     _tol(wl, got, want, "all-blocks")
 
 
-@pytest.mark.parametrize("wid", [1, 3, 2])
-def test_sparse_full_size_sampled(wid):
-    """Full-size workloads in the benchmark's launch configuration; sampled query blocks."""
-    wl = synth.WORKLOADS[wid]
-    L = C.layer(wid)
+@pytest.mark.parametrize("d,dtype", [(64, "bf16"), (128, "bf16"), (64, "f32")])
+def test_empty_rows_and_empty_pair_tiles(d, dtype):
+    # a caller-made mask where rows 0, 2, 3 and 6 keep nothing: tile 1 (rows 2, 3) and
+    # tile 3 (row 6 and the missing row 7) have no work at all; empty rows come out as
+    # zeros and the other rows are unaffected
+    wl = synth.custom_workload(3, 12, 12, 2, d, dtype, seed=40)   # N = 432, nB = 7
+    keep = {1: [0, 3], 4: [4, 6], 5: [1]}
+    got, want, _ = _custom_mask_run(wl, lambda bh, a: keep.get(a, []))
+    _tol(wl, got, want, "empty rows")
+    for a in (0, 2, 3, 6):
+        assert np.all(got[:, :, a * 64:min(a * 64 + 64, wl.N)] == 0.0), a
+
+
+def _sampled_check(wl, L, n_per_head, seed):
+    """Route and attend one layer in the benchmark's launch configuration, then compare
+    sampled query blocks (always the densest and the sparsest rows) with the oracle."""
     run = C.GpuRun(wl, L)
     g = run.mask_np()
     got = run.layer
@@ -162,7 +173,7 @@ def test_sparse_full_size_sampled(wid):
     torch.cuda.synchronize()
     assert run.status() == 0
     BH, nB = wl.B * wl.H, wl.nB
-    rows = C.sample_rows(g["row_ptr"], BH, nB, 6, seed=wid)
+    rows = C.sample_rows(g["row_ptr"], BH, nB, n_per_head, seed=seed)
     perm, _ = O.hilbert_perm(wl.T, wl.Hg, wl.Wg)
     max_err, sum_err, n = 0.0, 0.0, 0
     heads = sorted({bh for bh, _ in rows})
@@ -184,6 +195,18 @@ def test_sparse_full_size_sampled(wid):
     mean_err = sum_err / n
     print(f"{wl.name}: sampled {len(rows)} query blocks max-abs {max_err:.3e} mean-abs {mean_err:.3e}")
     assert max_err <= C.BF16_MAX_ABS and mean_err <= C.BF16_MEAN_ABS
+
+
+@pytest.mark.parametrize("wid", [1, 3, 2])
+def test_sparse_full_size_sampled(wid):
+    """Full-size workloads in the benchmark's launch configuration; sampled query blocks."""
+    _sampled_check(synth.WORKLOADS[wid], C.layer(wid), 6, wid)
+
+
+def test_sparse_at_largest_routable_shape():
+    """One head of 605,284 tokens (nB = 9458, the routing limit), 4,729 pair tiles."""
+    wl = C.largest_routable_workload()
+    _sampled_check(wl, synth.make_layer(wl), 10, 41)
 
 
 def test_dense_full_size_sampled_480p():

@@ -136,6 +136,18 @@ def test_route_720p_p_sweep(p):
     _check_route(wl, C.layer(2), p, wl.k_floor, order=2)
 
 
+def test_route_at_largest_routable_shape():
+    """nB = 9458, the largest block count routing supports (one more is rejected on the
+    host before any launch; see test_abi_cpu.py). The selection kernel runs with its
+    largest per-row shared-memory arena here."""
+    wl = C.largest_routable_workload()
+    assert wl.nB == 9458 and wl.N % 64 == 36
+    # at this nB the entry at a row's cut holds ~1e-4 of the row's mass, so the oracle's
+    # 1e-6 ambiguity band covers a few percent of the rows; mismatches outside the band
+    # must still be zero
+    _check_route(wl, synth.make_layer(wl), wl.p, wl.k_floor, order=2, max_amb_frac=5e-2)
+
+
 def test_hetero_heads_density_split():
     """Head-heterogeneity workload: the 20% flat heads (tau = 0.3) are far denser than the
     concentrated ones; their share of kept blocks is reported (0.40 with this generator)."""
