@@ -40,20 +40,57 @@ __device__ __forceinline__ void hilbert_cell(int m, uint32_t t, int* px, int* py
   *py = y;
 }
 
-// One CTA: enumerate the curve of the enclosing square in order, keep in-grid cells
-// (block-wide scan for their output slots) and write frame 0's order to perm[0, HW).
-__global__ void __launch_bounds__(1024) hilbert_frame_kernel(int m, int Hg, int Wg, int32_t* perm) {
+constexpr int kHilbertChunk = 1024;  // indices per pass: 4^5, one aligned 32 x 32 sub-square
+
+// Index of the first chunk (a multiple of 1024, so an aligned 32 x 32 sub-square) at or
+// after b that holds an in-grid cell. The 4^k indices from an index aligned to 4^k form
+// one aligned 2^k x 2^k sub-square (every level of the curve only reflects, swaps and
+// translates by multiples of the side), so a sub-square whose lower corner lies at or
+// beyond the frame is skipped whole, largest first. A wrong skip could only leave cells
+// out (perm is written at most Hg * Wg times), never write past the frame.
+
+__device__ uint64_t hilbert_next_chunk(uint64_t b, uint64_t total, int m, int Hg, int Wg) {
+  while (b < total) {
+    int k = m;
+    while (k > 5 && (b & ((1ull << (2 * k)) - 1)) != 0) --k;
+    int x, y;
+    hilbert_cell(m, static_cast<uint32_t>(b), &x, &y);
+    bool skipped = false;
+    for (; k >= 5; --k) {
+      const int corner = ~((1 << k) - 1);
+      if ((x & corner) >= Wg || (y & corner) >= Hg) {
+        b += 1ull << (2 * k);
+        skipped = true;
+        break;
+      }
+    }
+    if (!skipped) return b;
+  }
+  return total;
+}
+
+// One CTA: walk the curve of the enclosing square in order, 1024 indices at a time,
+// skipping sub-squares outside the frame, keep in-grid cells (block-wide scan for their
+// output slots) and write frame 0's order to perm[0, HW). The square has up to 4^16
+// cells, so indices are 64-bit; the work follows the frame's area, not the square's.
+__global__ void __launch_bounds__(kHilbertChunk) hilbert_frame_kernel(int m, int Hg, int Wg, int32_t* perm) {
   __shared__ int warp_tot[32];
   __shared__ int carry;
-  const uint32_t total = 1u << (2 * m);
+  __shared__ uint64_t next_base;
+  const uint64_t total = 1ull << (2 * m);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) carry = 0;
+  if (threadIdx.x == 0) {
+    carry = 0;
+    next_base = hilbert_next_chunk(0, total, m, Hg, Wg);
+  }
   __syncthreads();
-  for (uint32_t base = 0; base < total; base += blockDim.x) {
-    const uint32_t t = base + threadIdx.x;
+  while (true) {
+    const uint64_t base = next_base;
+    if (base >= total) break;
+    const uint64_t t = base + threadIdx.x;
     int x = 0, y = 0, valid = 0;
     if (t < total) {
-      hilbert_cell(m, t, &x, &y);
+      hilbert_cell(m, static_cast<uint32_t>(t), &x, &y);
       valid = (x < Wg && y < Hg) ? 1 : 0;
     }
     const uint32_t ballot = __ballot_sync(0xffffffffu, valid);
@@ -61,7 +98,7 @@ __global__ void __launch_bounds__(1024) hilbert_frame_kernel(int m, int Hg, int 
     if (lane == 0) warp_tot[warp] = __popc(ballot);
     __syncthreads();
     int before = 0, all = 0;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
+    for (int w = 0; w < kHilbertChunk / 32; ++w) {
       const int c = warp_tot[w];
       if (w < warp) before += c;
       all += c;
@@ -69,7 +106,10 @@ __global__ void __launch_bounds__(1024) hilbert_frame_kernel(int m, int Hg, int 
     const int pos = carry + before + in_warp;
     if (valid) perm[pos] = y * Wg + x;
     __syncthreads();
-    if (threadIdx.x == 0) carry += all;
+    if (threadIdx.x == 0) {
+      carry += all;
+      next_base = hilbert_next_chunk(base + kHilbertChunk, total, m, Hg, Wg);
+    }
     __syncthreads();
   }
 }
@@ -162,7 +202,7 @@ cudaError_t launch_hilbert_perm(const Dims& D, int T, int Hg, int Wg, int32_t* p
                                 cudaStream_t st) {
   int m = 0;
   while ((1 << m) < (Hg > Wg ? Hg : Wg)) ++m;
-  hilbert_frame_kernel<<<1, 1024, 0, st>>>(m, Hg, Wg, perm);
+  hilbert_frame_kernel<<<1, kHilbertChunk, 0, st>>>(m, Hg, Wg, perm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t HW = static_cast<int64_t>(Hg) * Wg;

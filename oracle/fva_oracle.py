@@ -100,6 +100,46 @@ def hilbert_perm(T: int, Hg: int, Wg: int):
     return perm, inv
 
 
+def hilbert_index(m: int, x, y) -> np.ndarray:
+    """Distance along the 2^m x 2^m Hilbert curve of each cell (x, y), int64.
+
+    A second construction of the curve above, read digit by digit from the top: at the
+    level of half-side s the cell lies in one of four quadrants, visited in the order
+    lower-left, upper-left, upper-right, lower-right, so it is preceded by
+    (quadrant number) * s^2 cells; the coordinates are then mapped into that quadrant's
+    own frame (lower-left: swap axes; lower-right: reflect about the anti-diagonal; the
+    upper quadrants keep their orientation) and the next level reads the next bit.
+    Works on frames far too large to enumerate (m up to 16)."""
+    x = np.asarray(x, dtype=np.int64).copy()
+    y = np.asarray(y, dtype=np.int64).copy()
+    d = np.zeros(np.broadcast(x, y).shape, dtype=np.int64)
+    for level in range(m - 1, -1, -1):
+        s = 1 << level
+        right = (x >> level) & 1
+        up = (y >> level) & 1
+        quadrant = np.where(right == 0, up, 3 - up)        # LL 0, UL 1, UR 2, LR 3
+        d += quadrant * s * s
+        low_x, low_y = x & (s - 1), y & (s - 1)
+        ll = quadrant == 0
+        lr = quadrant == 3
+        x = np.where(ll, low_y, np.where(lr, s - 1 - low_y, low_x))
+        y = np.where(ll, low_x, np.where(lr, s - 1 - low_x, low_y))
+    return d
+
+
+def hilbert_perm_by_index(T: int, Hg: int, Wg: int):
+    """hilbert_perm's order built the other way round: the frame's cells sorted by
+    hilbert_index on the enclosing square (no enumeration of the square's other cells)."""
+    m = hilbert_order_m(Hg, Wg)
+    yy, xx = np.divmod(np.arange(Hg * Wg, dtype=np.int64), Wg)
+    frame = (yy * Wg + xx)[np.argsort(hilbert_index(m, xx, yy), kind="stable")]
+    hw = Hg * Wg
+    perm = np.concatenate([t * hw + frame for t in range(T)]) if T > 0 else np.zeros(0, np.int64)
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(perm.size, dtype=np.int64)
+    return perm, inv
+
+
 # Variant of step 1 (a next step of the build, not the pages' own): a generalized
 # Hilbert curve that covers a W x H rectangle directly instead of the enclosing 2^m
 # square, following Jakub Cerveny's published generalized-Hilbert ("gilbert")

@@ -31,6 +31,32 @@ def test_hilbert_perm_exact(T, Hg, Wg):
     np.testing.assert_array_equal(inv.cpu().numpy(), want_i)
 
 
+# frames at the side limit (65536, an enclosing square of 4^16 cells), long strips and a
+# large near-square frame; the oracle sorts the cells by their index on the curve
+LARGE_FRAMES = [(1, 2, 65536), (1, 65536, 2), (2, 3, 40000), (1, 1, 65536), (1, 1500, 1300), (1, 4097, 5)]
+
+
+@pytest.mark.parametrize("T,Hg,Wg", LARGE_FRAMES)
+def test_hilbert_perm_exact_on_large_frames(T, Hg, Wg):
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import fva
+    s = fva.make_shape(1, 1, 64, T, Hg, Wg, "bf16")
+    N = T * Hg * Wg
+    perm = torch.empty(N, dtype=torch.int32, device="cuda")
+    inv = torch.empty(N, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fva.fva_hilbert_perm(s, perm, inv)
+    torch.cuda.synchronize()
+    want_p, want_i = O.hilbert_perm_by_index(T, Hg, Wg)
+    np.testing.assert_array_equal(perm.cpu().numpy(), want_p)
+    np.testing.assert_array_equal(inv.cpu().numpy(), want_i)
+    if Hg * Wg <= 200000:
+        fva.fva_curve_perm(s, fva.FVA_CURVE_RECT, perm, inv, st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        np.testing.assert_array_equal(perm.cpu().numpy(), O.rect_curve_perm(T, Hg, Wg)[0])
+
+
 @pytest.mark.parametrize("T,Hg,Wg", GRIDS + [(1, 40, 40), (2, 1, 77), (3, 33, 17)])
 def test_rect_curve_perm_exact(T, Hg, Wg):
     import torch

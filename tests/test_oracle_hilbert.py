@@ -118,3 +118,37 @@ def test_reorder_inverse_roundtrip():
     for i in (0, 5, N - 1):
         np.testing.assert_array_equal(xr[0, 2, i], x[0, perm[i], 2])
     np.testing.assert_array_equal(O.inverse_reorder(xr, perm), x)
+
+
+@pytest.mark.parametrize("m", [0, 1, 2, 3, 5, 7])
+def test_index_construction_inverts_the_recursive_curve(m):
+    # the digit-by-digit index of every cell of the recursive curve is its position on it
+    curve = O.hilbert_curve(m)
+    np.testing.assert_array_equal(O.hilbert_index(m, curve[:, 0], curve[:, 1]), np.arange(4 ** m))
+
+
+@pytest.mark.parametrize("T,Hg,Wg", [(1, 1, 1), (2, 3, 5), (1, 45, 80), (3, 30, 52), (1, 1, 200), (2, 97, 3),
+                                     (1, 64, 64)])
+def test_perm_by_index_equals_enumerated_perm(T, Hg, Wg):
+    a = O.hilbert_perm(T, Hg, Wg)
+    b = O.hilbert_perm_by_index(T, Hg, Wg)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_index_on_the_largest_square_walks_unit_steps():
+    # m = 16: consecutive indices along a sampled stretch are grid neighbours
+    m = 16
+    rng = np.random.default_rng(5)
+    side = 1 << m
+    for _ in range(4):
+        x0, y0 = (int(v) for v in rng.integers(0, side, 2))
+        d0 = int(O.hilbert_index(m, x0, y0))
+        xs, ys = np.meshgrid(np.arange(max(0, x0 - 40), min(side, x0 + 40)),
+                             np.arange(max(0, y0 - 40), min(side, y0 + 40)))
+        d = O.hilbert_index(m, xs.ravel(), ys.ravel())
+        near = np.argsort(d)
+        dd, xx, yy = d[near], xs.ravel()[near], ys.ravel()[near]
+        run = np.nonzero(np.diff(dd) == 1)[0]
+        assert run.size > 100 and d0 in dd
+        assert np.all(np.abs(xx[run + 1] - xx[run]) + np.abs(yy[run + 1] - yy[run]) == 1)
