@@ -312,9 +312,10 @@ def fva_sasa_augment(s, pooled_q, pooled_k, rank_of_head, budget, mask: Mask, wo
                      added=None, dev_status=None, stream=None):
     """Slack-aware augmentation of a routed mask in place (rank_of_head int32 [B*H] and
     budget int64 [n_ranks] on the device)."""
+    m = mask.c() if isinstance(mask, Mask) else mask
     _check("fva_sasa_augment", _lib.fva_sasa_augment(
         ctypes.byref(s), _ptr(pooled_q), _ptr(pooled_k), _ptr(rank_of_head), int(budget.shape[0]), _ptr(budget),
-        int(order), ctypes.byref(mask.c()), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        int(order), ctypes.byref(m), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _ptr(added), _ptr(dev_status), _stream(stream)))
 
 

@@ -16,6 +16,7 @@ layers all ranks processed in it.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import math
@@ -163,7 +164,6 @@ def rlb_report(costs: np.ndarray, BH: int, n_pairs: int, t_attn_ms: float, head_
     """Runtime Load Balancing on a virtual `ranks`-way head split of this layer: per-head
     load = its tiles' list lengths x the measured time per tile step on one GPU; P = the
     head's Q, K, V in and O out at the peer-copy rate; C = the planner's host time."""
-    import time
     from adaptive_block_sparse_hilbert_b200 import fva
     steps = costs.reshape(BH, n_pairs).sum(axis=1).astype(np.float64)
     unit = t_attn_ms / max(float(steps.sum()), 1.0)
@@ -390,7 +390,7 @@ def run_gpu(args):
     rank, world, local = dist_env()
     if world > 1:
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     else:
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
