@@ -18,7 +18,8 @@ Recipe (one layer of a video DiT, B=1, tokens in raster order n = t*Hg*Wg + y*Wg
 
 Values are drawn in float32 and then rounded to the workload's dtype (bf16 by
 round-to-nearest-even, or kept as fp32). The rounded values are what both the CUDA
-path and the oracle consume.
+path and the oracle consume. A batch of B > 1 (test cases only) stacks B such layers,
+each drawn from its own seed.
 
 The pages describe Wan2.x video DiTs at 720p/81 frames (21 latent frames x 3600
 tokens = 75,600 tokens); no trained weights are available, so these synthetic tensors
@@ -76,9 +77,11 @@ WORKLOADS = {
 P_SWEEP_720P = (0.8, 0.9, 0.95)
 
 
-def custom_workload(T, Hg, Wg, H, d, dtype="bf16", p=0.9, k_floor=4, seed=7, tau=("logU", 0.5, 4.0)):
-    """A workload of any grid/head shape with the same recipe (used for small test cases)."""
-    return Workload(f"custom_{T}x{Hg}x{Wg}_h{H}_d{d}_{dtype}", T, Hg, Wg, H, d, dtype, p, k_floor, tau, seed)
+def custom_workload(T, Hg, Wg, H, d, dtype="bf16", p=0.9, k_floor=4, seed=7, tau=("logU", 0.5, 4.0), B=1):
+    """A workload of any grid/head/batch shape with the same recipe (used for small test cases).
+    With B > 1 each batch entry is drawn as a layer of its own (see make_layer)."""
+    name = f"custom_{T}x{Hg}x{Wg}_h{H}_d{d}_{dtype}" + (f"_b{B}" if B > 1 else "")
+    return Workload(name, T, Hg, Wg, H, d, dtype, p, k_floor, tau, seed, B=B)
 
 
 # --------------------------------------------------------------------------------------
@@ -165,7 +168,15 @@ def _round(wl: Workload, x32: np.ndarray):
 
 
 def make_layer(wl: Workload, step: int = 0) -> Layer:
-    """Draw one layer (one denoising step for the multi-step drift workload)."""
+    """Draw one layer (one denoising step for the multi-step drift workload). With B > 1
+    every batch entry is a layer of its own (own field, tau, noise and V), drawn with the
+    seed 1000 * seed + b, so that the entries route differently."""
+    if wl.B > 1:
+        parts = [make_layer(dataclasses.replace(wl, B=1, seed=wl.seed * 1000 + b), step) for b in range(wl.B)]
+        cat = lambda xs: None if xs[0] is None else np.concatenate(xs, axis=0)  # noqa: E731
+        return Layer(wl, step, np.stack([x.tau for x in parts]), cat([x.q for x in parts]),
+                     cat([x.k for x in parts]), cat([x.v for x in parts]), cat([x.q_bits for x in parts]),
+                     cat([x.k_bits for x in parts]), cat([x.v_bits for x in parts]))
     if wl.steps > 1:
         # field of step s = (1 - a_s) field_{s-1} + a_s fresh_s ; step 0 is a fresh field
         field = None

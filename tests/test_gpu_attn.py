@@ -50,6 +50,8 @@ SMALL = [
     synth.custom_workload(1, 8, 8, 1, 64, "bf16", seed=34),              # a single block
     synth.custom_workload(2, 5, 7, 2, 64, "f32", seed=35),               # fp32 ragged
     synth.custom_workload(5, 16, 16, 2, 128, "bf16", seed=36, p=0.7, k_floor=1),
+    synth.custom_workload(3, 12, 17, 3, 128, "bf16", seed=42, B=2, p=0.8, k_floor=1),  # two batch entries
+    synth.custom_workload(3, 12, 17, 2, 64, "f32", seed=43, B=3, p=0.8, k_floor=1),    # fp32, three entries
 ]
 
 

@@ -9,11 +9,11 @@ from tests import _common as C
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("H,groups", [(5, 3), (4, 4), (6, 1), (7, None)])
-def test_pipelined_equals_one_shot(H, groups):
+@pytest.mark.parametrize("B,H,groups", [(1, 5, 3), (1, 4, 4), (1, 6, 1), (1, 7, None), (2, 5, 2)])
+def test_pipelined_equals_one_shot(B, H, groups):
     import torch
     from adaptive_block_sparse_hilbert_b200 import fva, pipeline
-    wl = synth.custom_workload(3, 10, 13, H, 128, "bf16", seed=81)
+    wl = synth.custom_workload(3, 10, 13, H, 128, "bf16", seed=81, B=B)
     L = synth.make_layer(wl)
     s = C.shape_of(wl)
     q, k, v = C.to_device(L)

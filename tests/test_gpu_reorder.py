@@ -84,6 +84,8 @@ SMALL = [
     synth.custom_workload(2, 9, 9, 2, 128, "bf16", seed=12),     # N = 162, tail of 34
     synth.custom_workload(1, 8, 8, 2, 128, "f32", seed=13),      # exactly one block
     synth.custom_workload(2, 5, 7, 2, 64, "f32", seed=14),       # N = 70
+    synth.custom_workload(3, 12, 17, 3, 128, "bf16", seed=15, B=2),  # two batch entries
+    synth.custom_workload(3, 5, 7, 2, 64, "f32", seed=16, B=3),     # three entries, fp32
 ]
 
 

@@ -62,6 +62,7 @@ SMALL = [
     synth.custom_workload(2, 9, 9, 2, 128, "bf16", seed=22, tau=("logU", 2.0, 6.0)),
     synth.custom_workload(2, 5, 7, 2, 64, "f32", seed=23),
     synth.custom_workload(4, 20, 20, 2, 64, "bf16", seed=24, tau=("logU", 0.2, 0.4)),
+    synth.custom_workload(3, 12, 17, 3, 64, "bf16", seed=27, B=2, p=0.8, k_floor=1),  # two batch entries
 ]
 
 

@@ -91,6 +91,7 @@ SMALL = [
     synth.custom_workload(4, 20, 20, 4, 64, "bf16", seed=71),
     synth.custom_workload(3, 10, 13, 3, 128, "bf16", seed=72, tau=("logU", 2.0, 6.0)),
     synth.custom_workload(2, 16, 16, 6, 64, "f32", seed=73),
+    synth.custom_workload(3, 12, 17, 3, 64, "bf16", seed=74, B=2, p=0.8, k_floor=1),  # two batch entries
 ]
 
 
