@@ -52,6 +52,8 @@ SMALL = [
     synth.custom_workload(5, 16, 16, 2, 128, "bf16", seed=36, p=0.7, k_floor=1),
     synth.custom_workload(3, 12, 17, 3, 128, "bf16", seed=42, B=2, p=0.8, k_floor=1),  # two batch entries
     synth.custom_workload(3, 12, 17, 2, 64, "f32", seed=43, B=3, p=0.8, k_floor=1),    # fp32, three entries
+    synth.custom_workload(2, 9, 11, 2, 32, "f32", seed=44, p=0.8, k_floor=1),          # fp32 d = 32
+    synth.custom_workload(2, 9, 11, 2, 128, "f32", seed=45, p=0.8, k_floor=1),         # fp32 d = 128
 ]
 
 
