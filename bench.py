@@ -311,9 +311,13 @@ def oracle_sample(wl, L, n_heads: int, rows_per_head: int, seed: int = 0):
         n_rows += len(rows)
     nh = len(heads)
     ms = 1e3 * (t_perm + (t_reorder + t_route) * wl.H / nh + t_attn * (wl.H * wl.nB) / n_rows)
-    sample = (f"{nh} of {wl.H} heads: reorder + pooling + full routing of each sampled head, attention on "
-              f"{rows_per_head} seeded query blocks per sampled head; time extrapolated linearly to all heads "
-              f"and all {wl.nB} query blocks (extrapolated)")
+    if nh == wl.H and n_rows == wl.H * wl.nB:
+        sample = (f"the full layer: reorder, pooling, routing and attention of all {wl.H} heads and all "
+                  f"{wl.nB} query blocks (no extrapolation)")
+    else:
+        sample = (f"{nh} of {wl.H} heads: reorder + pooling + full routing of each sampled head, attention on "
+                  f"{min(rows_per_head, wl.nB)} seeded query blocks per sampled head; time extrapolated linearly "
+                  f"to all heads and all {wl.nB} query blocks (extrapolated)")
     wall = t_perm + t_reorder + t_route + t_attn
     return ms, sample, wall
 
