@@ -96,8 +96,16 @@ class HostPipelinedLayer:
     SparseAttentionLayer on a shape with fewer heads, and the output equals the one-shot
     layer's bit for bit.
 
+    Consecutive forward() calls overlap too: a call's copy-in of a group waits only for the
+    previous call's compute of that group (the last reader of the group's input buffers),
+    and its compute waits for the previous call's copy-out of that group (the last reader of
+    its output buffer). So one layer's copies run during its neighbours' compute. The
+    caller's stream is never made to wait: call wait() (or synchronize) before reading
+    o_host, and do not overwrite a host input before the call that reads it has finished.
+
         layer = HostPipelinedLayer(shape, p=0.9, k_floor=4)   # ramp of head groups
         layer.forward(q_host, k_host, v_host, o_host)   # pinned CPU tensors, raster order
+        layer.wait()
     """
 
     def __init__(self, shape: fva.fva_shape, p: float, k_floor: int, groups=None,
@@ -133,36 +141,57 @@ class HostPipelinedLayer:
         self.s_in = torch.cuda.Stream(device=device)
         self.s_comp = torch.cuda.Stream(device=device)
         self.s_out = torch.cuda.Stream(device=device)
+        G = len(self.heads)
+        self.in_ready = [torch.cuda.Event() for _ in range(G)]    # group's inputs on the device
+        self.comp_done = [torch.cuda.Event() for _ in range(G)]   # group's compute finished
+        self.out_done = [torch.cuda.Event() for _ in range(G)]    # group's output in host memory
+        self.started = False
+        # the buffers (and each group's token order) were made on the current stream
+        made = torch.cuda.Event()
+        made.record(torch.cuda.current_stream())
+        for st in (self.s_in, self.s_comp, self.s_out):
+            st.wait_event(made)
 
     def forward(self, q_host, k_host, v_host, o_host):
-        """Enqueue the layer; returns the stream whose completion means o_host is written
-        (the caller's current stream is made to wait on it)."""
+        """Enqueue one layer and return the stream that copies its output out (see the
+        class notes: nothing is made to wait on it; wait() does that)."""
         s = self.shape
         row = s.H * s.d * self.esize
         rows = s.B * self.N
-        cur = torch.cuda.current_stream()
-        self.s_in.wait_stream(cur)
-        self.s_comp.wait_stream(cur)
-        self.s_out.wait_stream(cur)
-        ready = []
-        for (h0, n), qd, kd, vd in zip(self.heads, self.q_in, self.k_in, self.v_in):
+        for g, ((h0, n), qd, kd, vd) in enumerate(zip(self.heads, self.q_in, self.k_in, self.v_in)):
+            if self.started:
+                self.s_in.wait_event(self.comp_done[g])
             width = n * s.d * self.esize
             for dst, src in ((qd, q_host), (kd, k_host), (vd, v_host)):
                 fva.fva_copy_strided(dst, width, src[:, :, h0:h0 + n, :], row, width, rows, self.s_in)
-            ev = torch.cuda.Event()
-            ev.record(self.s_in)
-            ready.append(ev)
+            self.in_ready[g].record(self.s_in)
         for g, ((h0, n), layer) in enumerate(zip(self.heads, self.layers)):
-            self.s_comp.wait_event(ready[g])
+            self.s_comp.wait_event(self.in_ready[g])
+            if self.started:
+                self.s_comp.wait_event(self.out_done[g])
             layer.forward(self.q_in[g], self.k_in[g], self.v_in[g], self.o_out[g], self.s_comp)
-            done = torch.cuda.Event()
-            done.record(self.s_comp)
-            self.s_out.wait_event(done)
+            self.comp_done[g].record(self.s_comp)
+            self.s_out.wait_event(self.comp_done[g])
             width = n * s.d * self.esize
             fva.fva_copy_strided(o_host[:, :, h0:h0 + n, :], row, self.o_out[g], width, width, rows, self.s_out)
-        cur.wait_stream(self.s_out)
-        cur.wait_stream(self.s_comp)
+            self.out_done[g].record(self.s_out)
+        self.started = True
         return self.s_out
+
+    def after(self, stream=None):
+        """Make the layer's streams wait for the work already enqueued on `stream` (default:
+        the current stream), e.g. a timing event or a producer of the host inputs."""
+        st = torch.cuda.current_stream() if stream is None else stream
+        for side in (self.s_in, self.s_comp, self.s_out):
+            side.wait_stream(st)
+
+    def wait(self, stream=None):
+        """Make `stream` (default: the current stream) wait until every enqueued forward()
+        has finished, its output copied to host memory."""
+        st = torch.cuda.current_stream() if stream is None else stream
+        st.wait_stream(self.s_in)
+        st.wait_stream(self.s_comp)
+        st.wait_stream(self.s_out)
 
     def dev_status(self):
         """Largest device error code any group reported (0 = none)."""

@@ -29,6 +29,35 @@ def test_pipelined_equals_one_shot(B, H, groups):
     assert torch.equal(oh, o_ref.cpu())
 
 
+def test_consecutive_layers_overlap_without_races():
+    # three layers with different inputs enqueued back to back (their copies and compute
+    # overlap across calls), then one wait: each output equals its one-shot layer's
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import pipeline
+    wls = [synth.custom_workload(3, 10, 13, 5, 128, "bf16", seed=91 + i) for i in range(3)]
+    s = C.shape_of(wls[0])
+    one = pipeline.SparseAttentionLayer(s, wls[0].p, wls[0].k_floor)
+    pipe = pipeline.HostPipelinedLayer(s, wls[0].p, wls[0].k_floor, groups=3)
+    refs, hosts = [], []
+    for wl in wls:
+        q, k, v = C.to_device(synth.make_layer(wl))
+        o_ref = torch.empty_like(q)
+        one.forward(q, k, v, o_ref)
+        refs.append(o_ref.cpu())
+        hosts.append(tuple(t.cpu().pin_memory() for t in (q, k, v)) + (torch.zeros_like(q.cpu()).pin_memory(),))
+    torch.cuda.synchronize()
+    for rep in range(2):
+        for qh, kh, vh, oh in hosts:
+            pipe.forward(qh, kh, vh, oh)
+        pipe.wait()
+        torch.cuda.synchronize()
+        assert pipe.dev_status() == 0
+        for (_, _, _, oh), ref in zip(hosts, refs):
+            assert torch.equal(oh, ref), rep
+        for h in hosts:
+            h[3].zero_()
+
+
 def test_copy_strided_moves_a_head_slice():
     import torch
     from adaptive_block_sparse_hilbert_b200 import fva
