@@ -183,3 +183,38 @@ def test_lpt_order_and_union_costs():
     assert cost.tolist() == [3, 5, 1]
     assert O.lpt_order(cost).tolist() == [1, 0, 2]
     assert O.lpt_order(np.array([2, 5, 2, 5, 0])).tolist() == [1, 3, 0, 2, 4]
+
+
+# ---- ambiguity flags (they decide which GPU/oracle mask differences may be excused) ----
+
+def _logits_for(w):
+    """Logits whose softmax is w / sum(w): s = log w."""
+    return np.log(np.asarray(w, dtype=np.float64))
+
+
+@pytest.mark.parametrize("w,k_floor,want", [
+    ([0.5, 0.4 - 2e-7, 0.1 + 2e-7], 0, True),    # c_1 = p - 2e-7: the cut could move up
+    ([0.5, 0.4 + 2e-7, 0.1 - 2e-7], 0, True),    # c_1 = p + 2e-7: the cut could move down
+    ([0.5, 0.3, 0.2], 0, False),                 # c = 0.5, 0.8, 1.0: every mass 0.1 from p
+    ([0.5, 0.4 + 2e-7, 0.1 - 2e-7], 3, False),   # the floor (3 blocks) decides, not the mass
+])
+def test_mass_flag_only_when_the_cut_sits_within_the_band(w, k_floor, want):
+    s = _logits_for(w)
+    info = O.route_row(s, 0.9, k_floor)
+    amb = O.row_ambiguity(s, info, 0.9)
+    assert bool(amb["ambiguous_mass"]) == want
+    assert not amb["ambiguous_tie"]
+
+
+@pytest.mark.parametrize("s,want", [
+    ([1.0, 0.5, 0.5, -3.0], True),               # L = 2 and the 2nd/3rd logits tie: which one is kept is moot
+    ([1.0, 0.5, 0.5 - 5e-10, -3.0], True),       # closer than 1e-9 relative
+    ([1.0, 0.5, 0.5 - 5e-9, -3.0], False),       # 5e-9 apart: outside the band
+    ([1.0, -2.0, -3.0, -3.0], False),            # a tie, but away from the boundary (L = 1)
+])
+def test_tie_flag_only_at_the_boundary(s, want):
+    s = np.asarray(s, dtype=np.float64)
+    info = O.route_row(s, 0.5, 0)
+    amb = O.row_ambiguity(s, info, 0.5)
+    assert bool(amb["ambiguous_tie"]) == want
+    assert not amb["ambiguous_mass"]
