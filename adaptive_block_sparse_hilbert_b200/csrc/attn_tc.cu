@@ -14,7 +14,8 @@
 //     into a ring of stages), warp 5 issues tcgen05.mma (one thread), warps 0-3 own one
 //     query row per thread (TMEM lane) for the online softmax and the epilogue.
 //   * S = Q K^T (M=128, N=64, K=d, bf16 -> fp32) goes to one of two TMEM buffers; the
-//     softmax warps read it, write P back over it as packed bf16 and the MMA warp
+//     softmax warps read it, write P back over it as packed fp16 (bf16 in the bf16-V
+//     variant) and the MMA warp
 //     issues O += P V with P taken straight from TMEM (A operand) and V from shared
 //     memory (B operand, MN-major). O stays in TMEM until the epilogue.
 //   * O is rescaled only when a row maximum grows by more than 2^8 (log2 units), so

@@ -21,6 +21,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -371,16 +372,26 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------------- GPU arm
 
+def code_sha256(path: str) -> str:
+    """SHA-256 of a CUDA source's code: comments and blank lines removed, so that a record
+    keyed by it survives comment-only edits and lapses with any change to the code."""
+    with open(path, encoding="utf-8") as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln.strip()).encode()).hexdigest()
+
+
 def traffic_record(kernel_src: str):
-    """DRAM bytes per attention launch from the committed ncu summary, if it matches the source."""
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken on
+    the kernel's current code."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         rec = json.load(f)
-    sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
     r = rec.get("attn_bf16_kernel")
-    if not r or r.get("source_sha256") != sha:
+    if not r or r.get("code_sha256") != code_sha256(kernel_src):
         return None
     return r
 

@@ -52,3 +52,30 @@ def test_ramp_sizes(H):
     assert sizes[: 3] == [1, 2, 3][: len(sizes[:3])] or H < 6
     if H >= 10:
         assert sizes[:3] == [1, 2, 3] and sizes[-1] == 2
+
+
+def test_code_hash_ignores_comments_only(tmp_path):
+    base = "// header\n__global__ void k(int* x) {\n  x[0] = 1;  // store\n}\n"
+    a = tmp_path / "a.cu"
+    a.write_text(base)
+    b = tmp_path / "b.cu"
+    b.write_text("/* another\n   header */\n\n__global__ void k(int* x) {\n  x[0] = 1;\n}\n// tail\n")
+    c = tmp_path / "c.cu"
+    c.write_text(base.replace("x[0] = 1", "x[0] = 2"))
+    assert bench.code_sha256(str(a)) == bench.code_sha256(str(b))
+    assert bench.code_sha256(str(a)) != bench.code_sha256(str(c))
+
+
+def test_committed_traffic_record_scaling():
+    # the committed ncu DRAM record: per-launch traffic = the 480p capture scaled by tokens
+    # per head. Once the attention code changes the record lapses (the bench then reports
+    # traffic: null) until it is captured again.
+    import os
+    src = os.path.join(bench.ROOT, "adaptive_block_sparse_hilbert_b200", "csrc", "attn_tc.cu")
+    r = bench.traffic_record(src)
+    if r is None:
+        pytest.skip("the DRAM record was taken on other attention code; capture it again")
+    assert r["workload"] == "720p_21x45x80_h40_d128_bf16"
+    m = r["measured_bytes"]
+    assert r["traffic_bytes_per_launch"] == pytest.approx(
+        (m["dram__bytes_read.sum"] + m["dram__bytes_write.sum"]) * 75600 / 32760, rel=1e-3)
