@@ -39,3 +39,28 @@ def test_max_over_ranks_and_whole_job_value():
     for rank in range(world):
         assert res[rank][0] == 15.0 and res[rank][1] == 100.0
         assert res[rank][2] == pytest.approx(7.5)
+
+
+def _reference_arm(rank, world):
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload", "0",
+                          "--gpus", str(world), "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, env=env, timeout=300)
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    return out.returncode, [json.loads(ln) for ln in lines]
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    rc, lines = _reference_arm(1, 2)
+    assert rc == 0 and lines == []
+    rc, lines = _reference_arm(0, 2)
+    assert rc == 0 and len(lines) == 1
+    line = lines[0]
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["dtype"] == "f64"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    # default flags sample 4 of the 16 query blocks per head, so the time is extrapolated
+    assert line["cpu_baseline"]["sample"].endswith("(extrapolated)")

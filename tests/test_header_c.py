@@ -75,3 +75,18 @@ def test_header_is_strict_c99_and_host_entry_points_run_from_c(tmp_path):
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert run.returncode == 0, (run.returncode, run.stderr)
     assert run.stdout.strip() == "c abi ok"
+
+
+def test_header_compiles_as_cpp17():
+    cxx = shutil.which("g++") or shutil.which("c++")
+    if cxx is None:
+        pytest.skip("no C++ compiler")
+    import tempfile
+    with tempfile.TemporaryDirectory() as d:
+        src = os.path.join(d, "abi.cpp")
+        with open(src, "w") as f:
+            f.write('#include "fva.h"\nint main() { fva_shape s{}; return fva_num_tokens(&s) == -1 ? 0 : 1; }\n')
+        out = subprocess.run([cxx, "-std=c++17", "-Wall", "-Wextra", "-Werror", "-I", INCLUDE, "-fsyntax-only", src],
+                             capture_output=True, text=True)
+        assert out.returncode == 0, out.stderr
+
