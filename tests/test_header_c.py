@@ -17,6 +17,23 @@ PROGRAM = r"""
 #include <string.h>
 #include "fva.h"
 
+/* The calls of one layer, as the README shows them: compiled and linked here, never run
+   (the pointers would be device memory). */
+int example_layer(const void* q, const void* k, const void* v, void* o, void* qh, void* kh, void* vh, void* oh,
+                  double* pooled_q, double* pooled_k, int32_t* perm, int32_t* inv, fva_mask mask, void* ws,
+                  size_t ws_bytes, int32_t* status, fva_stream_t stream) {
+  fva_shape s = {1, 40, 128, 21, 45, 80, 64, FVA_BF16};
+  int rc = fva_hilbert_perm(&s, perm, inv, stream);
+  if (rc == FVA_OK) rc = fva_reorder(&s, q, qh, pooled_q, perm, FVA_FWD, stream);
+  if (rc == FVA_OK) rc = fva_reorder(&s, k, kh, pooled_k, perm, FVA_FWD, stream);
+  if (rc == FVA_OK) rc = fva_reorder(&s, v, vh, NULL, perm, FVA_FWD_F16, stream);
+  if (rc == FVA_OK)
+    rc = fva_route(&s, NULL, NULL, pooled_q, pooled_k, 0.9, 4, FVA_ORDER_HEAD_LPT, &mask, ws, ws_bytes, status, stream);
+  if (rc == FVA_OK) rc = fva_sparse_attn(&s, qh, kh, vh, FVA_F16, &mask, oh, 0.0f, status, stream);
+  if (rc == FVA_OK) rc = fva_reorder(&s, oh, o, NULL, perm, FVA_INV, stream);
+  return rc;
+}
+
 int main(void) {
   fva_shape s = {1, 40, 128, 21, 45, 80, 64, FVA_BF16}; /* 720p: 75,600 tokens, nB = 1182 */
   if (fva_num_tokens(&s) != 75600) return 1;
