@@ -7,7 +7,8 @@
 // never fewer than k_floor blocks.
 //
 // Kernels (all float64 where a value decides the mask):
-//   route_scores_kernel   S = pooled_q pooled_k^T / sqrt(d), register-tiled DFMA GEMM
+//   route_scores_kernel   S = pooled_q pooled_k^T / sqrt(d), a GEMM on the FP64 tensor-core
+//                         MMA (mma.sync m8n8k4.f64)
 //   route_select_kernel   one warp per row: softmax, bucket refinement to the cut,
 //                         exact (logit desc, index asc) order inside the last bucket,
 //                         kept bitmask, kept count, per-tile union cost
@@ -24,94 +25,93 @@ namespace fva {
 // Block logits
 // ---------------------------------------------------------------------------------
 constexpr int kST = 128;  // output tile (rows and columns)
-constexpr int kSK = 8;    // d-chunk staged per step (d is a multiple of 8)
-constexpr int kSP = kST + 2;  // padded row: transposed stores spread over banks, rows stay 16-B aligned
 
-// grid: (ceil(nB/128), ceil(nB/128), B*H); 256 threads in a 16 x 16 grid, each an 8 x 8
-// block of logits: rows {4 ty + i, 64 + 4 ty + i} and columns {4 tx + j, 64 + 4 tx + j},
-// i, j < 4, so every shared-memory operand read is a 16-byte pair and a warp's B reads are
-// contiguous. 16 operand loads per 64 DFMA per chunk column.
+constexpr int kDK = 16;       // d-chunk staged per step (every supported d is a multiple of 16)
+constexpr int kDP = kDK + 4;  // padded row (doubles): a half-warp's fragment loads hit 32 banks
+
+__device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(d0), "+d"(d1)
+               : "d"(a), "d"(b));
+}
+
+// grid: (ceil(nB/128), ceil(nB/128), B*H); 8 warps as 2 (rows) x 4 (columns), each a
+// 64 x 32 block of logits in 8 x 4 MMA tiles of 8 x 8 (lane (g, t) holds A[g][t], B[t][g]
+// and C[g][2t], C[g][2t+1] of a tile).
 __global__ void __launch_bounds__(256, 1) route_scores_kernel(const double* __restrict__ pq,
                                                               const double* __restrict__ pk,
                                                               double* __restrict__ S, int nB, int d,
                                                               double sqrt_d) {
-  __shared__ __align__(16) double As[kSK][kSP];
-  __shared__ __align__(16) double Bs[kSK][kSP];
+  __shared__ __align__(16) double As[kST][kDP];
+  __shared__ __align__(16) double Bs[kST][kDP];
   const int bh = blockIdx.z;
   const int a0 = blockIdx.y * kST, b0 = blockIdx.x * kST;
   const double* Q = pq + static_cast<int64_t>(bh) * nB * d;
   const double* K = pk + static_cast<int64_t>(bh) * nB * d;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  double acc[8][8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wm = warp & 1, wn = warp >> 1;
+  const int g = lane >> 2, t = lane & 3;
+  double acc[8][4][2];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int mi = 0; mi < 8; ++mi)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+    for (int ni = 0; ni < 4; ++ni) acc[mi][ni][0] = acc[mi][ni][1] = 0.0;
 
-  // each thread stages four consecutive d-elements of one row of each tile
-  const int lr = threadIdx.x >> 1;        // 0..127: row within the tile
-  const int lc = (threadIdx.x & 1) * 4;   // 0 or 4: d offset within the chunk
+  // each thread stages eight consecutive d-elements of one row of each tile
+  const int lr = threadIdx.x >> 1;
+  const int lc = (threadIdx.x & 1) * 8;
   const int ga = a0 + lr, gb = b0 + lr;
-  // the next chunk is loaded into registers while the current one is multiplied
-  double2 q0 = make_double2(0.0, 0.0), q1 = q0, k0 = q0, k1 = q0;
+  double2 qv[4], kv[4];
   auto fetch = [&](int i0) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      qv[j] = make_double2(0.0, 0.0);
+      kv[j] = qv[j];
+    }
     if (ga < nB) {
       const double2* src = reinterpret_cast<const double2*>(Q + static_cast<int64_t>(ga) * d + i0 + lc);
-      q0 = src[0];
-      q1 = src[1];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) qv[j] = src[j];
     }
     if (gb < nB) {
       const double2* src = reinterpret_cast<const double2*>(K + static_cast<int64_t>(gb) * d + i0 + lc);
-      k0 = src[0];
-      k1 = src[1];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) kv[j] = src[j];
     }
   };
   fetch(0);
-  for (int i0 = 0; i0 < d; i0 += kSK) {
-    As[lc][lr] = q0.x;
-    As[lc + 1][lr] = q0.y;
-    As[lc + 2][lr] = q1.x;
-    As[lc + 3][lr] = q1.y;
-    Bs[lc][lr] = k0.x;
-    Bs[lc + 1][lr] = k0.y;
-    Bs[lc + 2][lr] = k1.x;
-    Bs[lc + 3][lr] = k1.y;
+  for (int i0 = 0; i0 < d; i0 += kDK) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      *reinterpret_cast<double2*>(&As[lr][lc + 2 * j]) = qv[j];
+      *reinterpret_cast<double2*>(&Bs[lr][lc + 2 * j]) = kv[j];
+    }
     __syncthreads();
-    if (i0 + kSK < d) fetch(i0 + kSK);
+    if (i0 + kDK < d) fetch(i0 + kDK);
 #pragma unroll
-    for (int c = 0; c < kSK; ++c) {
-      double av[8], bv[8];
+    for (int kk = 0; kk < kDK; kk += 4) {
+      double af[8], bf[4];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const double2 a01 = *reinterpret_cast<const double2*>(&As[c][h * 64 + ty * 4]);
-        const double2 a23 = *reinterpret_cast<const double2*>(&As[c][h * 64 + ty * 4 + 2]);
-        const double2 b01 = *reinterpret_cast<const double2*>(&Bs[c][h * 64 + tx * 4]);
-        const double2 b23 = *reinterpret_cast<const double2*>(&Bs[c][h * 64 + tx * 4 + 2]);
-        av[4 * h] = a01.x;
-        av[4 * h + 1] = a01.y;
-        av[4 * h + 2] = a23.x;
-        av[4 * h + 3] = a23.y;
-        bv[4 * h] = b01.x;
-        bv[4 * h + 1] = b01.y;
-        bv[4 * h + 2] = b23.x;
-        bv[4 * h + 3] = b23.y;
-      }
+      for (int mi = 0; mi < 8; ++mi) af[mi] = As[wm * 64 + mi * 8 + g][kk + t];
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int ni = 0; ni < 4; ++ni) bf[ni] = Bs[wn * 32 + ni * 8 + g][kk + t];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fma(av[i], bv[j], acc[i][j]);
+      for (int mi = 0; mi < 8; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) dmma_8x8x4(acc[mi][ni][0], acc[mi][ni][1], af[mi], bf[ni]);
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int a = a0 + (i >> 2) * 64 + ty * 4 + (i & 3);
+  for (int mi = 0; mi < 8; ++mi) {
+    const int a = a0 + wm * 64 + mi * 8 + g;
     if (a >= nB) continue;
     double* dst = S + (static_cast<int64_t>(bh) * nB + a) * nB;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int b = b0 + (j >> 2) * 64 + tx * 4 + (j & 3);
-      if (b < nB) dst[b] = acc[i][j] / sqrt_d;
+    for (int ni = 0; ni < 4; ++ni) {
+      const int b = b0 + wn * 32 + ni * 8 + 2 * t;
+      if (b < nB) dst[b] = acc[mi][ni][0] / sqrt_d;
+      if (b + 1 < nB) dst[b + 1] = acc[mi][ni][1] / sqrt_d;
     }
   }
 }
