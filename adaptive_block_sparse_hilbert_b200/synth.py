@@ -89,15 +89,34 @@ def custom_workload(T, Hg, Wg, H, d, dtype="bf16", p=0.9, k_floor=4, seed=7, tau
 # --------------------------------------------------------------------------------------
 
 
-def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """float32 array -> uint16 bf16 bit patterns (round-to-nearest-even; inputs finite)."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
-    rounding = ((u >> 16) & 1) + np.uint32(0x7FFF)
-    return ((u + rounding) >> 16).astype(np.uint16)
+def f32_to_bf16_bits(x: np.ndarray, chunk: int = 1 << 20) -> np.ndarray:
+    """float32 array -> uint16 bf16 bit patterns (round-to-nearest-even; inputs finite).
+    Works through the array in chunks that stay in cache."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.reshape(-1).view(np.uint32)
+    out = np.empty(u.size, dtype=np.uint16)
+    tmp = np.empty(min(chunk, max(u.size, 1)), dtype=np.uint32)
+    for s in range(0, u.size, chunk):
+        c = u[s:s + chunk]
+        t = tmp[:c.size]
+        np.right_shift(c, 16, out=t)
+        np.bitwise_and(t, 1, out=t)  # lowest kept bit: ties go to even
+        t += np.uint32(0x7FFF)
+        t += c
+        t >>= 16
+        out[s:s + c.size] = t
+    return out.reshape(x.shape)
 
 
-def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
-    return (b.astype(np.uint32) << 16).view(np.float32)
+def bf16_bits_to_f32(b: np.ndarray, chunk: int = 1 << 20) -> np.ndarray:
+    b = np.ascontiguousarray(b, dtype=np.uint16)
+    flat = b.reshape(-1)
+    out = np.empty(flat.size, dtype=np.uint32)
+    for s in range(0, flat.size, chunk):
+        o = out[s:s + chunk]
+        o[:] = flat[s:s + chunk]
+        o <<= 16
+    return out.view(np.float32).reshape(b.shape)
 
 
 # --------------------------------------------------------------------------------------

@@ -172,3 +172,36 @@ def largest_routable_workload():
     nB = 9458 (a ragged tail of 36), d = 64. Heads drawn with tau in logU(2, 2.5) give a
     density near 0.18 with row lengths from a few dozen to thousands of blocks."""
     return synth.custom_workload(1, 778, 778, 1, 64, "bf16", seed=41, tau=("logU", 2.0, 2.5))
+
+
+def sampled_attention_errors(run, wl, L, g, n_per_head, seed, curve=0):
+    """Attend with the run's routed mask `g` (from run.mask_np()) and compare sampled query
+    blocks of every head -- seeded ones plus each head's densest, sparsest and ragged tail
+    rows -- with the oracle's attention over the same kept blocks. Returns (max-abs error,
+    mean-abs error, query blocks compared)."""
+    torch = torch_dev()
+    run.layer.attend()
+    torch.cuda.synchronize()
+    assert run.status() == 0
+    BH, nB = wl.B * wl.H, wl.nB
+    rows = sample_rows(g["row_ptr"], BH, nB, n_per_head, seed=seed)
+    perm, _ = (O.rect_curve_perm if curve == 1 else O.hilbert_perm)(wl.T, wl.Hg, wl.Wg)
+    max_err, sum_err, n = 0.0, 0.0, 0
+    oh = run.layer.oh
+    for bh in sorted({bh for bh, _ in rows}):
+        b, h = divmod(bh, wl.H)
+        qh = O.reorder(L.q[b:b + 1, :, h:h + 1], perm)[0, 0]
+        kh = O.reorder(L.k[b:b + 1, :, h:h + 1], perm)[0, 0]
+        vh = O.reorder(L.v[b:b + 1, :, h:h + 1], perm)[0, 0]
+        for (b2, a) in rows:
+            if b2 != bh:
+                continue
+            keys = O.block_keys(O.row_list(g["row_ptr"], g["col_idx"], bh * nB + a), wl.N)
+            lo, hi = a * 64, min(a * 64 + 64, wl.N)
+            want = O.attention_rows(qh[lo:hi], kh, vh, keys, 1.0 / np.sqrt(wl.d))
+            gv = oh[b, h, lo:hi].float().cpu().numpy().astype(np.float64)
+            diff = np.abs(gv - want)
+            max_err = max(max_err, float(diff.max()))
+            sum_err += float(diff.sum())
+            n += diff.size
+    return max_err, sum_err / n, len(rows)

@@ -170,35 +170,9 @@ def _sampled_check(wl, L, n_per_head, seed):
     """Route and attend one layer in the benchmark's launch configuration, then compare
     sampled query blocks (always the densest and the sparsest rows) with the oracle."""
     run = C.GpuRun(wl, L)
-    g = run.mask_np()
-    got = run.layer
-    import torch
-    got.attend()
-    torch.cuda.synchronize()
-    assert run.status() == 0
-    BH, nB = wl.B * wl.H, wl.nB
-    rows = C.sample_rows(g["row_ptr"], BH, nB, n_per_head, seed=seed)
-    perm, _ = O.hilbert_perm(wl.T, wl.Hg, wl.Wg)
-    max_err, sum_err, n = 0.0, 0.0, 0
-    heads = sorted({bh for bh, _ in rows})
-    for bh in heads:
-        qh = O.reorder(L.q[:, :, bh:bh + 1], perm)[0, 0]
-        kh = O.reorder(L.k[:, :, bh:bh + 1], perm)[0, 0]
-        vh = O.reorder(L.v[:, :, bh:bh + 1], perm)[0, 0]
-        for (b2, a) in rows:
-            if b2 != bh:
-                continue
-            keys = O.block_keys(O.row_list(g["row_ptr"], g["col_idx"], bh * nB + a), wl.N)
-            lo, hi = a * 64, min(a * 64 + 64, wl.N)
-            want = O.attention_rows(qh[lo:hi], kh, vh, keys, 1.0 / np.sqrt(wl.d))
-            gv = got.oh[0, bh, lo:hi].float().cpu().numpy().astype(np.float64)
-            diff = np.abs(gv - want)
-            max_err = max(max_err, float(diff.max()))
-            sum_err += float(diff.sum())
-            n += diff.size
-    mean_err = sum_err / n
-    print(f"{wl.name}: sampled {len(rows)} query blocks max-abs {max_err:.3e} mean-abs {mean_err:.3e}")
-    assert max_err <= C.BF16_MAX_ABS and mean_err <= C.BF16_MEAN_ABS
+    mx, mean, n_rows = C.sampled_attention_errors(run, wl, L, run.mask_np(), n_per_head, seed)
+    print(f"{wl.name}: sampled {n_rows} query blocks max-abs {mx:.3e} mean-abs {mean:.3e}")
+    assert mx <= C.BF16_MAX_ABS and mean <= C.BF16_MEAN_ABS
 
 
 @pytest.mark.parametrize("wid", [1, 3, 2])

@@ -132,9 +132,15 @@ def test_route_full_size(wid):
 
 
 @pytest.mark.parametrize("p", [0.8, 0.95])
-def test_route_720p_p_sweep(p):
+def test_route_and_attend_720p_p_sweep(p):
+    """The 720p layer at the other two p of the sweep: every mask row against the oracle,
+    then the attention output on sampled query blocks (densest, sparsest, tail, seeded)."""
     wl = synth.WORKLOADS[2]
-    _check_route(wl, C.layer(2), p, wl.k_floor, order=2)
+    L = C.layer(2)
+    run, g, _ = _check_route(wl, L, p, wl.k_floor, order=2)
+    mx, mean, n_rows = C.sampled_attention_errors(run, wl, L, g, 3, seed=int(p * 100))
+    print(f"{wl.name} p={p}: sampled {n_rows} query blocks max-abs {mx:.3e} mean-abs {mean:.3e}")
+    assert mx <= C.BF16_MAX_ABS and mean <= C.BF16_MEAN_ABS
 
 
 def test_route_at_largest_routable_shape():

@@ -2,9 +2,13 @@
 host owns every device allocation, a service that allocates nothing after start-up).
 
 It must give exactly the mask, tiles and work list of fva_route with a caller
-workspace, on two calls in a row (the second call reuses the library's fixed scratch
-array with the first call's contents still in it), and must turn away shapes whose
-scratch does not fit before doing any work. The file is named to be collected last.
+workspace, on every call: two workloads in a row (the second call finds the first call's
+larger scratch contents still in the library's fixed array), and the same inputs again
+into a mask that already holds the previous result. It must turn away shapes whose
+scratch does not fit before doing any work.
+
+The file name sorts after every other test file, so pytest collects it last: a GPU run
+that stops at its first failure has then run all the other GPU tests before this one.
 """
 import ctypes
 
@@ -17,10 +21,13 @@ from tests import _common as C
 pytestmark = pytest.mark.gpu
 
 
-def _noalloc_mask(run, p, k_floor, use_pooled):
+def _noalloc_mask(run, p, k_floor, use_pooled, m=None):
+    """Route through fva_route_noalloc into mask `m` (a fresh one when None); returns the
+    mask's contents and the mask."""
     import torch
     from adaptive_block_sparse_hilbert_b200 import fva
-    m = fva.Mask.allocate(run.shape)
+    if m is None:
+        m = fva.Mask.allocate(run.shape)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     lay = run.layer
     if use_pooled:
@@ -37,7 +44,7 @@ def _noalloc_mask(run, p, k_floor, use_pooled):
         "tile_col": m.tile_col[: int(tp[-1])].cpu().numpy().astype(np.int64),
         "tile_cost": m.tile_cost.cpu().numpy().astype(np.int64),
         "worklist": m.worklist.cpu().numpy().astype(np.int64),
-    }
+    }, m
 
 
 def test_noalloc_route_matches_workspace_route_twice():
@@ -50,9 +57,11 @@ def test_noalloc_route_matches_workspace_route_twice():
         L = synth.make_layer(wl)
         run = C.GpuRun(wl, L, p=p, k_floor=kf)          # fva_route with a caller workspace
         want = run.mask_np()
-        got = _noalloc_mask(run, p, kf, use_pooled)      # the same inputs, no workspace
+        got, m = _noalloc_mask(run, p, kf, use_pooled)   # the same inputs, no workspace
+        again, _ = _noalloc_mask(run, p, kf, use_pooled, m)  # once more, into the filled mask
         for key in want:
             np.testing.assert_array_equal(got[key], want[key], err_msg=f"{wl.name}: {key}")
+            np.testing.assert_array_equal(again[key], want[key], err_msg=f"{wl.name}: {key} (repeat)")
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
