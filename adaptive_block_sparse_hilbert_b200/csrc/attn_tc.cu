@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                      const __grid_constant__ CUtensorMap tmv, __nv_bfloat16* __restrict__ out,
                      const int32_t* __restrict__ tile_ptr, const int32_t* __restrict__ tile_col,
-                     const int32_t* __restrict__ worklist, int N, int nB, int nPairs, float scale_log2,
+                     const int32_t* __restrict__ worklist, int slot0, int ntiles, int N, int nB, int nPairs, float scale_log2,
                      uint64_t kWaitLimitNs, uint32_t diag_flags, int32_t* dev_status, int64_t* cta_trace) {
   using Cfg = AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -95,12 +95,23 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   AttnBars<D>& bar = *reinterpret_cast<AttnBars<D>*>(smem + Cfg::kSmemData);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = DENSE ? static_cast<int>(blockIdx.x) : worklist[blockIdx.x];
+  const int slot = static_cast<int>(blockIdx.x) + slot0;  // position in the work list
+  int tile = DENSE ? static_cast<int>(blockIdx.x) : worklist[slot];
+  // a work-list entry that names no tile is reported; its CTA then runs an empty list on
+  // tile 0 and writes nothing
+  const bool tile_ok = DENSE || (tile >= 0 && tile < ntiles);
+  if (!tile_ok) {
+    if (threadIdx.x == 0) report(dev_status, FVA_DEVERR_BAD_LIST);
+    tile = 0;
+  }
   const int bh = tile / nPairs;
   const int t = tile - bh * nPairs;
   int n_iter, list_base;
   if (DENSE) {
     n_iter = nB;
+    list_base = 0;
+  } else if (!tile_ok) {
+    n_iter = 0;
     list_base = 0;
   } else {
     list_base = tile_ptr[tile];
@@ -394,7 +405,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             dst[cc * 4 + q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         }
       }
-      if (n_iter == 0 && grow < N) {
+      if (n_iter == 0 && grow < N && tile_ok) {
         for (int q = 0; q < D / 8; ++q) dst[q] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
@@ -409,7 +420,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   if (cta_trace != nullptr && threadIdx.x == 0) {
     uint32_t smid;
     asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-    int64_t* rec = cta_trace + 4 * static_cast<int64_t>(blockIdx.x);
+    int64_t* rec = cta_trace + 4 * static_cast<int64_t>(DENSE ? static_cast<int>(blockIdx.x) : slot);
     rec[0] = smid;
     rec[1] = n_iter;
     rec[2] = static_cast<int64_t>(t_start);
@@ -468,41 +479,44 @@ static bool make_map(CUtensorMap* map, const void* base, int64_t BH, int64_t N, 
 
 template <int D, bool DENSE, bool VF16>
 static cudaError_t launch_attn_t(const Dims& Dm, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                                 const fva_mask* m, void* o, float scale_log2, int32_t* dev_status, cudaStream_t st) {
+                                 const fva_mask* m, void* o, float scale_log2, int first_slot, int n_slots,
+                                 int32_t* dev_status, cudaStream_t st) {
   const size_t smem = attn_smem_bytes<D>();
   cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<D, DENSE, VF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(Dm.tiles);
+  const unsigned grid = static_cast<unsigned>(DENSE ? Dm.tiles : n_slots);
+  if (grid == 0) return cudaSuccess;
   attn_bf16_kernel<D, DENSE, VF16><<<grid, kAttnThreads, smem, st>>>(
       mq, mk, mv, static_cast<__nv_bfloat16*>(o), DENSE ? nullptr : m->tile_ptr, DENSE ? nullptr : m->tile_col,
-      DENSE ? nullptr : m->worklist, static_cast<int>(Dm.N), static_cast<int>(Dm.nB), static_cast<int>(Dm.nPairs),
+      DENSE ? nullptr : m->worklist, DENSE ? 0 : first_slot, static_cast<int>(Dm.tiles), static_cast<int>(Dm.N), static_cast<int>(Dm.nB), static_cast<int>(Dm.nPairs),
       scale_log2, attn_wait_limit_ns(), attn_diag_flags(), dev_status, g_cta_trace);
   return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t launch_attn_d(const Dims& Dm, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                                 bool v_f16, const fva_mask* m, bool dense, void* o, float scale_log2,
-                                 int32_t* dev_status, cudaStream_t st) {
+                                 bool v_f16, const fva_mask* m, bool dense, void* o, float scale_log2, int first_slot,
+                                 int n_slots, int32_t* dev_status, cudaStream_t st) {
   if (v_f16) {
-    return dense ? launch_attn_t<D, true, true>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st)
-                 : launch_attn_t<D, false, true>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st);
+    return dense ? launch_attn_t<D, true, true>(Dm, mq, mk, mv, m, o, scale_log2, 0, 0, dev_status, st)
+                 : launch_attn_t<D, false, true>(Dm, mq, mk, mv, m, o, scale_log2, first_slot, n_slots, dev_status, st);
   }
-  return dense ? launch_attn_t<D, true, false>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st)
-               : launch_attn_t<D, false, false>(Dm, mq, mk, mv, m, o, scale_log2, dev_status, st);
+  return dense ? launch_attn_t<D, true, false>(Dm, mq, mk, mv, m, o, scale_log2, 0, 0, dev_status, st)
+               : launch_attn_t<D, false, false>(Dm, mq, mk, mv, m, o, scale_log2, first_slot, n_slots, dev_status, st);
 }
 
 cudaError_t launch_attn_bf16(const Dims& Dm, const void* q, const void* k, const void* v, bool v_f16,
-                             const fva_mask* m, bool dense, void* o, float scale, int32_t* dev_status,
-                             cudaStream_t st) {
+                             const fva_mask* m, bool dense, void* o, float scale, int64_t first_slot, int64_t n_slots,
+                             int32_t* dev_status, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, Dm.BH, Dm.N, Dm.d, false) || !make_map(&mk, k, Dm.BH, Dm.N, Dm.d, false) ||
       !make_map(&mv, v, Dm.BH, Dm.N, Dm.d, v_f16))
     return cudaErrorInvalidValue;
   const float scale_log2 = scale * 1.4426950408889634f;
-  if (Dm.d == 128) return launch_attn_d<128>(Dm, mq, mk, mv, v_f16, m, dense, o, scale_log2, dev_status, st);
-  return launch_attn_d<64>(Dm, mq, mk, mv, v_f16, m, dense, o, scale_log2, dev_status, st);
+  const int fs = static_cast<int>(first_slot), ns = static_cast<int>(n_slots);
+  if (Dm.d == 128) return launch_attn_d<128>(Dm, mq, mk, mv, v_f16, m, dense, o, scale_log2, fs, ns, dev_status, st);
+  return launch_attn_d<64>(Dm, mq, mk, mv, v_f16, m, dense, o, scale_log2, fs, ns, dev_status, st);
 }
 
 }  // namespace fva

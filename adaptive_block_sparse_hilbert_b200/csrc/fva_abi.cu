@@ -182,6 +182,7 @@ static int check_mask_outputs(const Dims& D, const fva_mask* m) {
     return FVA_ERR_INVALID_ARG;
   if (m->capacity < D.BH * D.nB * D.nB || m->tile_capacity < D.BH * D.nPairs * D.nB) return FVA_ERR_CAPACITY;
   if (D.BH * D.nB * D.nB > 0x7fffffffLL) return FVA_ERR_UNSUPPORTED_SHAPE;
+  if (m->logits && !aligned16(m->logits)) return FVA_ERR_ALIGNMENT;
   return FVA_OK;
 }
 
@@ -219,6 +220,7 @@ int fva_route(const fva_shape* s, const void* q_bhnd_dev, const void* k_bhnd_dev
     pq = wq;
     pk = wk;
   }
+  if (mask->logits) rs.scores = mask->logits;  // the logits go to the caller's buffer
   return cuda_status(launch_route(D, pq, pk, p, k_floor, order, mask, rs, dev_status, stream));
 }
 
@@ -242,8 +244,9 @@ int fva_sasa_augment(const fva_shape* s, const double* pooled_q_dev, const doubl
                      const fva_mask* mask, void* workspace_dev, size_t workspace_bytes, int64_t* added_dev,
                      int32_t* dev_status, fva_stream_t stream) {
   Dims D;
-  if (!s || !pooled_q_dev || !pooled_k_dev || !rank_of_head_dev || !budget_dev || !workspace_dev)
-    return FVA_ERR_INVALID_ARG;
+  if (!s || !rank_of_head_dev || !budget_dev || !workspace_dev) return FVA_ERR_INVALID_ARG;
+  if (!mask) return FVA_ERR_INVALID_ARG;
+  if (!mask->logits && (!pooled_q_dev || !pooled_k_dev)) return FVA_ERR_INVALID_ARG;
   if (n_ranks < 1 || n_ranks > FVA_SASA_MAX_RANKS) return FVA_ERR_INVALID_ARG;
   if (order != FVA_ORDER_NATURAL && order != FVA_ORDER_LPT && order != FVA_ORDER_HEAD_LPT) return FVA_ERR_INVALID_ARG;
   if (!make_dims(s, &D)) return FVA_ERR_UNSUPPORTED_SHAPE;
@@ -252,7 +255,8 @@ int fva_sasa_augment(const fva_shape* s, const double* pooled_q_dev, const doubl
   if (rc != FVA_OK) return rc;
   const size_t base = route_scratch_layout(D, 0, nullptr, nullptr, nullptr, nullptr, true);
   if (workspace_bytes < base + sasa_extra_bytes(D)) return FVA_ERR_WORKSPACE;
-  if (!aligned16(workspace_dev) || !aligned16(pooled_q_dev) || !aligned16(pooled_k_dev)) return FVA_ERR_ALIGNMENT;
+  if (!aligned16(workspace_dev)) return FVA_ERR_ALIGNMENT;
+  if (!mask->logits && (!aligned16(pooled_q_dev) || !aligned16(pooled_k_dev))) return FVA_ERR_ALIGNMENT;
   RouteScratch rs;
   route_scratch_layout(D, 0, workspace_dev, &rs, nullptr, nullptr, true);
   return cuda_status(launch_sasa(D, pooled_q_dev, pooled_k_dev, rank_of_head_dev, n_ranks, budget_dev, order, mask,
@@ -292,22 +296,30 @@ int fva_build_tiles(const fva_shape* s, const fva_mask* mask, int order, void* w
 }
 
 static int attn_common(const fva_shape* s, const void* q, const void* k, const void* v, int v_dtype,
-                       const fva_mask* m, void* o, float scale, bool dense, int32_t* dev_status, fva_stream_t stream) {
+                       const fva_mask* m, void* o, float scale, bool dense, int64_t first_slot, int64_t n_slots,
+                       bool whole, int32_t* dev_status, fva_stream_t stream) {
   Dims D;
   if (!s || !q || !k || !v || !o) return FVA_ERR_INVALID_ARG;
   if (!make_dims(s, &D)) return FVA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FVA_ERR_ALIGNMENT;
   if (o == q || o == k || o == v) return FVA_ERR_INVALID_ARG;
+  if (whole) {
+    first_slot = 0;
+    n_slots = D.tiles;
+  }
+  if (first_slot < 0 || n_slots < 0 || first_slot + n_slots > D.tiles) return FVA_ERR_INVALID_ARG;
   if (!(scale > 0.0f)) scale = 1.0f / sqrtf(static_cast<float>(D.d));
   if (s->dtype == FVA_BF16) {
     if (v_dtype != FVA_BF16 && v_dtype != FVA_F16) return FVA_ERR_INVALID_ARG;
     if (D.d != 64 && D.d != 128) return FVA_ERR_UNSUPPORTED_SHAPE;
     if (!dense && (!m || !m->tile_ptr || !m->tile_col || !m->worklist)) return FVA_ERR_INVALID_ARG;
     if (!attn_cta_trace_fits(D.tiles)) return FVA_ERR_CAPACITY;
-    return cuda_status(launch_attn_bf16(D, q, k, v, v_dtype == FVA_F16, m, dense, o, scale, dev_status, stream));
+    return cuda_status(launch_attn_bf16(D, q, k, v, v_dtype == FVA_F16, m, dense, o, scale, first_slot, n_slots,
+                                        dev_status, stream));
   }
   if (v_dtype != FVA_F32) return FVA_ERR_INVALID_ARG;
   if (D.d != 32 && D.d != 64 && D.d != 128) return FVA_ERR_UNSUPPORTED_SHAPE;
+  if (!whole) return FVA_ERR_UNSUPPORTED_SHAPE;  // the fp32 path reads the CSR, not the work list
   if (!dense && (!m || !m->row_ptr || !m->col_idx)) return FVA_ERR_INVALID_ARG;
   return cuda_status(launch_attn_f32(D, static_cast<const float*>(q), static_cast<const float*>(k),
                                      static_cast<const float*>(v), dense ? nullptr : m->row_ptr,
@@ -316,12 +328,19 @@ static int attn_common(const fva_shape* s, const void* q, const void* k, const v
 
 int fva_sparse_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev, int v_dtype,
                     const fva_mask* mask, void* o_dev, float scale, int32_t* dev_status, fva_stream_t stream) {
-  return attn_common(s, q_dev, k_dev, v_dev, v_dtype, mask, o_dev, scale, false, dev_status, stream);
+  return attn_common(s, q_dev, k_dev, v_dev, v_dtype, mask, o_dev, scale, false, 0, 0, true, dev_status, stream);
+}
+
+int fva_sparse_attn_range(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev, int v_dtype,
+                          const fva_mask* mask, void* o_dev, float scale, int64_t first_slot, int64_t n_slots,
+                          int32_t* dev_status, fva_stream_t stream) {
+  return attn_common(s, q_dev, k_dev, v_dev, v_dtype, mask, o_dev, scale, false, first_slot, n_slots, false,
+                     dev_status, stream);
 }
 
 int fva_dense_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev, int v_dtype,
                    void* o_dev, float scale, int32_t* dev_status, fva_stream_t stream) {
-  return attn_common(s, q_dev, k_dev, v_dev, v_dtype, nullptr, o_dev, scale, true, dev_status, stream);
+  return attn_common(s, q_dev, k_dev, v_dev, v_dtype, nullptr, o_dev, scale, true, 0, 0, true, dev_status, stream);
 }
 
 }  // extern "C"

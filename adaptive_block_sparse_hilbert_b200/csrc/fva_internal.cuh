@@ -56,9 +56,10 @@ cudaError_t launch_csr_to_bits(const Dims& D, const fva_mask* m, uint32_t* bits,
 cudaError_t launch_tiles_from_bits(const Dims& D, const fva_mask* m, int order, const RouteScratch& ws,
                                    const int32_t* row_cnt, int write_rows, int32_t* dev_status, cudaStream_t st);
 
+// Sparse: the CTAs of work-list slots [first_slot, first_slot + n_slots); dense: every tile.
 cudaError_t launch_attn_bf16(const Dims& D, const void* q, const void* k, const void* v, bool v_f16,
-                             const fva_mask* m, bool dense, void* o, float scale,
-                             int32_t* dev_status, cudaStream_t st);
+                             const fva_mask* m, bool dense, void* o, float scale, int64_t first_slot,
+                             int64_t n_slots, int32_t* dev_status, cudaStream_t st);
 uint64_t attn_wait_limit_ns();
 uint32_t attn_diag_flags();
 void set_attn_diagnostics(uint64_t wait_limit_ns, uint32_t flags);

@@ -257,22 +257,27 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4& v) {
 // MODE 1: inverse permute [B,H,N,d] -> [B,N,H,d]
 // MODE 2: pool only, input already [B,H,N,d]
 // MODE 3: forward permute with the output converted bf16 -> fp16
-// One CTA per (block a, head h, batch b); VPR = 16-byte vectors per (token, head) row.
-// Every thread keeps one vector column and loads all of its rows before storing any,
-// so a CTA has its whole 64-row block in flight.
-template <typename T, int MODE, bool POOL, int VPR>
+// One CTA per (block a, group of G adjacent heads, batch b); VPR = 16-byte vectors per
+// (token, head) row. The G heads of one token are adjacent in [B,N,H,d], so a token's
+// G * VPR vectors are one contiguous run: short rows (d * sizeof(T) < 256 B) are moved
+// G heads at a time and every CTA moves 64 rows of 256 B or more. Every thread keeps one
+// vector column and loads all of its rows before storing any, so a CTA has its whole
+// 64-row block in flight.
+template <typename T, int MODE, bool POOL, int VPR, int G>
 __global__ void __launch_bounds__(kReorderThreads) reorder_kernel(
     const uint8_t* __restrict__ x_in, uint8_t* __restrict__ x_out, double* __restrict__ pooled,
     const int32_t* __restrict__ perm, int N, int H) {
   constexpr int EPV = 16 / sizeof(T);          // elements per 16-byte vector
-  constexpr int RPP = kReorderThreads / VPR;   // rows per pass
+  constexpr int VPT = VPR * G;                 // vectors per token (its G heads)
+  constexpr int RPP = kReorderThreads / VPT;   // rows per pass
   constexpr int NPASS = (kBlock + RPP - 1) / RPP;
   constexpr int64_t kRowBytes = VPR * 16;
   constexpr int kWidth = VPR * EPV;            // = d
-  __shared__ double red[POOL ? RPP * kWidth : 1];
-  const int a = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int v = threadIdx.x % VPR;
-  const int r0 = threadIdx.x / VPR;
+  __shared__ double red[POOL ? RPP * kWidth * G : 1];
+  const int a = blockIdx.x, h0 = blockIdx.y * G, b = blockIdx.z;
+  const int v = threadIdx.x % VPT;             // vector within the token's G heads
+  const int g = v / VPR, vc = v % VPR;         // its head within the group, its column
+  const int r0 = threadIdx.x / VPT;
   const int row_lo = a * kBlock;
   const int n_valid = min(kBlock, N - row_lo);
   uint4 buf[NPASS];
@@ -281,13 +286,13 @@ __global__ void __launch_bounds__(kReorderThreads) reorder_kernel(
     const int r = r0 + ps * RPP;
     if (r < n_valid) {
       const int i = row_lo + r;
-      const uint8_t* src;
+      const uint4* src;
       if (MODE == 0 || MODE == 3) {
-        src = x_in + ((static_cast<int64_t>(b) * N + perm[i]) * H + h) * kRowBytes;
+        src = reinterpret_cast<const uint4*>(x_in + ((static_cast<int64_t>(b) * N + perm[i]) * H + h0) * kRowBytes) + v;
       } else {
-        src = x_in + ((static_cast<int64_t>(b) * H + h) * N + i) * kRowBytes;
+        src = reinterpret_cast<const uint4*>(x_in + ((static_cast<int64_t>(b) * H + h0 + g) * N + i) * kRowBytes) + vc;
       }
-      buf[ps] = __ldg(reinterpret_cast<const uint4*>(src) + v);
+      buf[ps] = __ldg(src);
     }
   }
   double acc[POOL ? EPV : 1];
@@ -301,50 +306,67 @@ __global__ void __launch_bounds__(kReorderThreads) reorder_kernel(
     if (r < n_valid) {
       const int i = row_lo + r;
       if (MODE != 2) {
-        uint8_t* dst;
+        uint4* dst;
         if (MODE == 0 || MODE == 3) {
-          dst = x_out + ((static_cast<int64_t>(b) * H + h) * N + i) * kRowBytes;
+          dst = reinterpret_cast<uint4*>(x_out + ((static_cast<int64_t>(b) * H + h0 + g) * N + i) * kRowBytes) + vc;
         } else {
-          dst = x_out + ((static_cast<int64_t>(b) * N + perm[i]) * H + h) * kRowBytes;
+          dst = reinterpret_cast<uint4*>(x_out + ((static_cast<int64_t>(b) * N + perm[i]) * H + h0) * kRowBytes) + v;
         }
-        reinterpret_cast<uint4*>(dst)[v] = (MODE == 3) ? bf16x8_to_f16x8(buf[ps]) : buf[ps];
+        *dst = (MODE == 3) ? bf16x8_to_f16x8(buf[ps]) : buf[ps];
       }
       if (POOL) add_vec<T>(acc, buf[ps]);
     }
   }
   if (POOL) {
 #pragma unroll
-    for (int e = 0; e < EPV; ++e) red[r0 * kWidth + v * EPV + e] = acc[e];
+    for (int e = 0; e < EPV; ++e) red[r0 * (G * kWidth) + v * EPV + e] = acc[e];
     __syncthreads();
-    // column sums over the RPP partial rows, fixed order
-    for (int c = threadIdx.x; c < kWidth; c += kReorderThreads) {
-      double s = 0.0;
+    // column sums over the RPP partial rows, fixed order; column c of the group is column
+    // c % d of head h0 + c / d
+    for (int c = threadIdx.x; c < G * kWidth; c += kReorderThreads) {
+      double sum = 0.0;
 #pragma unroll 8
-      for (int r = 0; r < RPP; ++r) s += red[r * kWidth + c];
-      pooled[((static_cast<int64_t>(b) * H + h) * gridDim.x + a) * kWidth + c] = s / static_cast<double>(n_valid);
+      for (int r = 0; r < RPP; ++r) sum += red[r * (G * kWidth) + c];
+      const int hh = h0 + c / kWidth;
+      pooled[((static_cast<int64_t>(b) * H + hh) * gridDim.x + a) * kWidth + (c % kWidth)] =
+          sum / static_cast<double>(n_valid);
     }
   }
 }
 
-template <typename T, int VPR>
-static cudaError_t launch_reorder_v(const Dims& D, const void* x_in, void* x_out, double* pooled,
+template <typename T, int VPR, int G>
+static cudaError_t launch_reorder_g(const Dims& D, const void* x_in, void* x_out, double* pooled,
                                     const int32_t* perm, int mode, cudaStream_t st) {
-  const dim3 grid(static_cast<unsigned>(D.nB), static_cast<unsigned>(D.H), static_cast<unsigned>(D.B));
+  const dim3 grid(static_cast<unsigned>(D.nB), static_cast<unsigned>(D.H / G), static_cast<unsigned>(D.B));
   const uint8_t* in = static_cast<const uint8_t*>(x_in);
   uint8_t* out = static_cast<uint8_t*>(x_out);
   const int N = static_cast<int>(D.N), H = static_cast<int>(D.H);
   if (mode == 0 && pooled) {
-    reorder_kernel<T, 0, true, VPR><<<grid, kReorderThreads, 0, st>>>(in, out, pooled, perm, N, H);
+    reorder_kernel<T, 0, true, VPR, G><<<grid, kReorderThreads, 0, st>>>(in, out, pooled, perm, N, H);
   } else if (mode == 0) {
-    reorder_kernel<T, 0, false, VPR><<<grid, kReorderThreads, 0, st>>>(in, out, nullptr, perm, N, H);
+    reorder_kernel<T, 0, false, VPR, G><<<grid, kReorderThreads, 0, st>>>(in, out, nullptr, perm, N, H);
   } else if (mode == 1) {
-    reorder_kernel<T, 1, false, VPR><<<grid, kReorderThreads, 0, st>>>(in, out, nullptr, perm, N, H);
+    reorder_kernel<T, 1, false, VPR, G><<<grid, kReorderThreads, 0, st>>>(in, out, nullptr, perm, N, H);
   } else if (mode == 3) {
-    reorder_kernel<T, 3, false, VPR><<<grid, kReorderThreads, 0, st>>>(in, out, nullptr, perm, N, H);
+    reorder_kernel<T, 3, false, VPR, G><<<grid, kReorderThreads, 0, st>>>(in, out, nullptr, perm, N, H);
   } else {
-    reorder_kernel<T, 2, true, VPR><<<grid, kReorderThreads, 0, st>>>(in, nullptr, pooled, nullptr, N, H);
+    reorder_kernel<T, 2, true, VPR, G><<<grid, kReorderThreads, 0, st>>>(in, nullptr, pooled, nullptr, N, H);
   }
   return cudaGetLastError();
+}
+
+// Heads moved together: enough that a token's group spans 16 vectors (256 B), and a
+// divisor of H.
+template <typename T, int VPR>
+static cudaError_t launch_reorder_v(const Dims& D, const void* x_in, void* x_out, double* pooled,
+                                    const int32_t* perm, int mode, cudaStream_t st) {
+  if constexpr (VPR == 4) {
+    if (D.H % 4 == 0) return launch_reorder_g<T, VPR, 4>(D, x_in, x_out, pooled, perm, mode, st);
+  }
+  if constexpr (VPR <= 8) {
+    if (D.H % 2 == 0) return launch_reorder_g<T, VPR, 2>(D, x_in, x_out, pooled, perm, mode, st);
+  }
+  return launch_reorder_g<T, VPR, 1>(D, x_in, x_out, pooled, perm, mode, st);
 }
 
 template <typename T>

@@ -10,9 +10,9 @@
 // A rank's budget goes to the skipped (row, block) entries of its heads with the largest
 // routing importance P_ab = softmax_b(s_ab), ties to the lower head, query block and key
 // block. On the device:
-//   1. the block logits are recomputed and, for every skipped entry, replaced in place by a
-//      64-bit key that orders like P (the bits of the positive double P, plus one; kept
-//      entries get 0);
+//   1. the block logits (exported by the routing pass, or recomputed) give, for every
+//      skipped entry, a 64-bit key that orders like P (the bits of the positive double P,
+//      plus one; kept entries get 0);
 //   2. an exact radix select fixes, 8 bits per pass from the top, the key tau_r of each
 //      rank's budget-th largest entry (per-CTA shared histograms, one picking step per pass);
 //   3. entries equal to tau_r are shared out in (head, query block) order, lower key block
@@ -35,15 +35,17 @@ __device__ __forceinline__ int rank_of_row(const int32_t* rank_of, int64_t row, 
   return (r >= 0 && r < R) ? r : -1;
 }
 
-// per row: row maximum, Z = sum exp(s - max), then keys over the logits; counts candidates
-__global__ void __launch_bounds__(256) sasa_keys_kernel(double* __restrict__ scores, const uint32_t* __restrict__ bits,
-                                                        int64_t rows, int nB, int nWords,
-                                                        const int32_t* __restrict__ rank_of, int R,
+// per row: row maximum, Z = sum exp(s - max), then one key per entry; counts candidates.
+// `logits` and `keys_out` may be the same array (the keys then replace the logits: every
+// lane writes only the entries it has just read, after the row's reductions).
+__global__ void __launch_bounds__(256) sasa_keys_kernel(const double* logits, uint64_t* keys_out,
+                                                        const uint32_t* __restrict__ bits, int64_t rows, int nB,
+                                                        int nWords, const int32_t* __restrict__ rank_of, int R,
                                                         unsigned long long* total, int32_t* dev_status) {
   const int lane = threadIdx.x & 31;
   const int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= rows) return;
-  double* s = scores + r * nB;
+  const double* s = logits + r * nB;
   const int rk = rank_of_row(rank_of, r, nB, R);
   if (rk < 0 && lane == 0 && (r % nB) == 0) report(dev_status, FVA_DEVERR_BAD_LIST);
   double mx = -INFINITY;
@@ -52,7 +54,7 @@ __global__ void __launch_bounds__(256) sasa_keys_kernel(double* __restrict__ sco
   double z = 0.0;
   for (int b = lane; b < nB; b += 32) z += exp(s[b] - mx);
   z = warp_sum_d(z);
-  uint64_t* key = reinterpret_cast<uint64_t*>(s);
+  uint64_t* key = keys_out + r * nB;
   unsigned cnt = 0;
   for (int b = lane; b < nB; b += 32) {
     const bool kept = (bits[r * nWords + (b >> 5)] >> (b & 31)) & 1u;
@@ -244,10 +246,16 @@ cudaError_t launch_sasa(const Dims& D, const double* pq, const double* pk, const
   const unsigned row_grid = static_cast<unsigned>((D.rows + 7) / 8);
   cudaError_t e = cudaMemsetAsync(hist, 0, kSasaMaxRanks * kSasaBins * 4, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(total, 0, kSasaMaxRanks * 8, st);
-  if (e == cudaSuccess) e = launch_route_scores(D, pq, pk, ws.scores, st);
+  // the block logits: exported by the routing pass (mask->logits), else recomputed
+  const double* logits = m->logits;
+  if (!logits && e == cudaSuccess) {
+    e = launch_route_scores(D, pq, pk, ws.scores, st);
+    logits = ws.scores;
+  }
   if (e == cudaSuccess) e = launch_csr_to_bits(D, m, ws.bits, dev_status, st);
   if (e != cudaSuccess) return e;
-  sasa_keys_kernel<<<row_grid, 256, 0, st>>>(ws.scores, ws.bits, D.rows, nB, nWords, rank_of, R, total, dev_status);
+  sasa_keys_kernel<<<row_grid, 256, 0, st>>>(logits, reinterpret_cast<uint64_t*>(ws.scores), ws.bits, D.rows, nB,
+                                             nWords, rank_of, R, total, dev_status);
   sasa_init_kernel<<<1, kSasaMaxRanks, 0, st>>>(budget, R, total, prefix, pmask, need, added);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

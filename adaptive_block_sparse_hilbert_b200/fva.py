@@ -54,7 +54,8 @@ class fva_shape(ctypes.Structure):
 class fva_mask(ctypes.Structure):
     _fields_ = [("row_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p), ("capacity", ctypes.c_int64),
                 ("head_kept", ctypes.c_void_p), ("tile_ptr", ctypes.c_void_p), ("tile_col", ctypes.c_void_p),
-                ("tile_capacity", ctypes.c_int64), ("tile_cost", ctypes.c_void_p), ("worklist", ctypes.c_void_p)]
+                ("tile_capacity", ctypes.c_int64), ("tile_cost", ctypes.c_void_p), ("worklist", ctypes.c_void_p),
+                ("logits", ctypes.c_void_p)]
 
 
 class fva_rlb_move(ctypes.Structure):
@@ -103,6 +104,7 @@ def _load():
         "fva_build_tiles": (i32, [S, M, i32, P, sz, P, P]),
         "fva_route_noalloc": (i32, [S, P, P, P, P, dbl, i32, i32, M, P, P]),
         "fva_sparse_attn": (i32, [S, P, P, P, i32, M, P, flt, P, P]),
+        "fva_sparse_attn_range": (i32, [S, P, P, P, i32, M, P, flt, i64, i64, P, P]),
         "fva_dense_attn": (i32, [S, P, P, P, i32, P, flt, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -118,7 +120,7 @@ EXPORTED = (
     "fva_tile_capacity", "fva_route_workspace_bytes", "fva_tiles_workspace_bytes", "fva_hilbert_perm", "fva_reorder",
     "fva_pool", "fva_route", "fva_build_tiles", "fva_sparse_attn", "fva_dense_attn", "fva_route_noalloc",
     "fva_set_cta_trace", "fva_rlb_plan", "fva_curve_perm", "fva_sasa_budgets", "fva_sasa_workspace_bytes",
-    "fva_sasa_augment", "fva_copy_strided",
+    "fva_sasa_augment", "fva_copy_strided", "fva_sparse_attn_range",
 )
 
 
@@ -233,9 +235,10 @@ class Mask:
     tile_col: torch.Tensor
     tile_cost: torch.Tensor
     worklist: torch.Tensor
+    logits: torch.Tensor | None = None  # optional float64 [B*H, nB, nB]: the exported block logits
 
     @staticmethod
-    def allocate(s: fva_shape, device="cuda") -> "Mask":
+    def allocate(s: fva_shape, device="cuda", logits: bool = False) -> "Mask":
         B, H = s.B, s.H
         nB = fva_num_blocks(s)
         tiles = fva_num_tiles(s)
@@ -248,12 +251,14 @@ class Mask:
             tile_col=torch.empty(fva_tile_capacity(s), **i32),
             tile_cost=torch.empty(tiles, **i32),
             worklist=torch.empty(tiles, **i32),
+            logits=torch.empty((B * H, nB, nB), dtype=torch.float64, device=device) if logits else None,
         )
 
     def c(self) -> fva_mask:
         return fva_mask(self.row_ptr.data_ptr(), self.col_idx.data_ptr(), self.col_idx.numel(),
                         self.head_kept.data_ptr(), self.tile_ptr.data_ptr(), self.tile_col.data_ptr(),
-                        self.tile_col.numel(), self.tile_cost.data_ptr(), self.worklist.data_ptr())
+                        self.tile_col.numel(), self.tile_cost.data_ptr(), self.worklist.data_ptr(),
+                        None if self.logits is None else self.logits.data_ptr())
 
 
 # ------------------------------------------------------------------------------ entry points
@@ -335,6 +340,16 @@ def fva_sparse_attn(s, q, k, v, mask: Mask, o, scale=0.0, dev_status=None, strea
     vd = _dtype_code(v) if v_dtype is None else int(v_dtype)
     _check("fva_sparse_attn", _lib.fva_sparse_attn(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), vd, ctypes.byref(m),
                                                    _ptr(o), float(scale), _ptr(dev_status), _stream(stream)))
+
+
+def fva_sparse_attn_range(s, q, k, v, mask: Mask, o, first_slot, n_slots, scale=0.0, dev_status=None, stream=None,
+                          v_dtype=None):
+    """The tiles at work-list positions [first_slot, first_slot + n_slots) only."""
+    m = mask.c() if isinstance(mask, Mask) else mask
+    vd = _dtype_code(v) if v_dtype is None else int(v_dtype)
+    _check("fva_sparse_attn_range", _lib.fva_sparse_attn_range(
+        ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), vd, ctypes.byref(m), _ptr(o), float(scale), int(first_slot),
+        int(n_slots), _ptr(dev_status), _stream(stream)))
 
 
 def fva_dense_attn(s, q, k, v, o, scale=0.0, dev_status=None, stream=None, v_dtype=None):

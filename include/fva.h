@@ -108,6 +108,15 @@ typedef struct fva_shape {
  *                                      key_block*4 | (row 2t keeps it) | (row 2t+1 keeps it)<<1
  *   tile_cost int32 [B*H*nPairs]       number of entries of each tile (its work)
  *   worklist  int32 [B*H*nPairs]       tile ids in launch order (see FVA_ORDER_*)
+ *   logits    float64 [B*H, nB, nB]    OPTIONAL (NULL: not used). When set, fva_route writes
+ *                                      every row's block logits s_ab here: the importance
+ *                                      order of the row's key blocks (larger logit first,
+ *                                      lower block on ties) and, through the row softmax,
+ *                                      their importances. fva_sasa_augment then reads them
+ *                                      instead of recomputing them ([aixai] "Sparse-routing
+ *                                      frontend": the one routing pass yields both the
+ *                                      per-head density and the importance order that the
+ *                                      augmentation uses). 16-byte aligned.
  */
 typedef struct fva_mask {
   int32_t* row_ptr;
@@ -119,6 +128,7 @@ typedef struct fva_mask {
   int64_t tile_capacity;
   int32_t* tile_cost;
   int32_t* worklist;
+  double* logits;
 } fva_mask;
 
 FVA_API const char* fva_status_string(int status);
@@ -220,7 +230,8 @@ FVA_API int fva_pool(const fva_shape* s, const void* x_bhnd_dev, double* pooled_
  * or, when both are NULL, q_bhnd_dev/k_bhnd_dev (Hilbert-ordered, pooled here into the
  * workspace; needs fva_route_workspace_bytes(s, 1)).
  * Outputs: every array of *mask (row_ptr, col_idx, head_kept, tile_ptr, tile_col,
- * tile_cost, worklist); mask->capacity >= fva_mask_capacity(s) and
+ * tile_cost, worklist), and mask->logits when it is not NULL (the block logits, which
+ * otherwise stay in the workspace); mask->capacity >= fva_mask_capacity(s) and
  * mask->tile_capacity >= fva_tile_capacity(s) are required. order is a FVA_ORDER_*.
  * 0 < p <= 1, k_floor >= 0.
  */
@@ -259,6 +270,21 @@ FVA_API int fva_build_tiles(const fva_shape* s, const fva_mask* mask, int order,
 FVA_API int fva_sparse_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev,
                             int v_dtype, const fva_mask* mask, void* o_dev, float scale, int32_t* dev_status,
                             fva_stream_t stream);
+
+/*
+ * Part of a sparse attention launch: the tiles at work-list positions
+ * [first_slot, first_slot + n_slots) of mask->worklist (bf16 inputs only; fp32 inputs give
+ * FVA_ERR_UNSUPPORTED_SHAPE). Output rows of the other tiles are left untouched, so
+ * consecutive ranges that together cover the list give fva_sparse_attn's result; a range
+ * may also leave tiles out (with FVA_ORDER_HEAD_LPT a head's tiles are consecutive in the
+ * list, so a head that another GPU computes can be skipped: [aixai] "Runtime Load
+ * Balancing (RLB)", migration of a heavy head to a less loaded rank).
+ * 0 <= first_slot, 0 <= n_slots, first_slot + n_slots <= fva_num_tiles(s), else
+ * FVA_ERR_INVALID_ARG; n_slots == 0 enqueues nothing. Other arguments as fva_sparse_attn.
+ */
+FVA_API int fva_sparse_attn_range(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev,
+                                  int v_dtype, const fva_mask* mask, void* o_dev, float scale, int64_t first_slot,
+                                  int64_t n_slots, int32_t* dev_status, fva_stream_t stream);
 
 /* Dense attention (every block kept): the in-house density-1 reference. Same layouts. */
 FVA_API int fva_dense_attn(const fva_shape* s, const void* q_dev, const void* k_dev, const void* v_dev,
@@ -336,7 +362,11 @@ FVA_API int fva_rlb_plan(const double* head_load_ms, int n_heads, int n_ranks, d
  * rows of the heads with rank_of_head_dev[h] == r. A rank with fewer skipped entries than
  * its budget gets all of them. The mask is rewritten in place: CSR, head_kept, tile lists
  * and the work list in `order` (FVA_ORDER_*).
- *   pooled_q_dev / pooled_k_dev: float64 [B, H, nB, d] as for fva_route;
+ *   pooled_q_dev / pooled_k_dev: float64 [B, H, nB, d] as for fva_route; both may be NULL
+ *     when mask->logits is set, and are then not read;
+ *   mask->logits: when not NULL, the block logits fva_route wrote there for this mask (the
+ *     same pooled Q/K); the augmentation takes the importances from them instead of
+ *     recomputing the logits (one float64 read of B*H*nB*nB values instead of a GEMM);
  *   rank_of_head_dev: int32 [B*H] device, values in [0, n_ranks) (others: FVA_DEVERR_BAD_LIST
  *     in dev_status, and the head is left unchanged); n_ranks in [1, FVA_SASA_MAX_RANKS];
  *   budget_dev: int64 [n_ranks] device (negative counts as 0);

@@ -164,3 +164,25 @@ def test_copy_strided_argument_checks():
     assert L.fva_copy_strided(1024, 16, 2048, 8, 16, 1, None) == fva.FVA_ERR_INVALID_ARG   # width > src pitch
     assert L.fva_copy_strided(1024, 16, 2048, 16, 16, -1, None) == fva.FVA_ERR_INVALID_ARG
     assert L.fva_copy_strided(1024, 16, 2048, 16, 16, 0, None) == fva.FVA_OK               # nothing to move
+
+
+def test_sparse_attn_range_host_checks():
+    """fva_sparse_attn_range turns away slot ranges outside the work list, and fp32 inputs,
+    before anything is enqueued (the pointers here are never dereferenced)."""
+    s = fva.make_shape(1, 2, 128, 2, 16, 16, "bf16")    # nB = 8, 4 tiles per head, 8 tiles
+    assert fva.fva_num_tiles(s) == 8
+    m = fva.fva_mask(16, 16, 10, 16, 16, 16, 10, 16, 16)
+    p = ctypes.c_void_p(256)
+    o = ctypes.c_void_p(512)
+
+    def rng(first, n, shape=s, vd=fva.FVA_F16):
+        return fva.call_raw("fva_sparse_attn_range", ctypes.byref(shape), p, p, p, vd, ctypes.byref(m), o,
+                            ctypes.c_float(0.0), first, n, None, None)
+    assert rng(-1, 2) == fva.FVA_ERR_INVALID_ARG
+    assert rng(0, -1) == fva.FVA_ERR_INVALID_ARG
+    assert rng(5, 4) == fva.FVA_ERR_INVALID_ARG       # past the 8 tiles
+    assert rng(9, 0) == fva.FVA_ERR_INVALID_ARG
+    f32 = fva.make_shape(1, 2, 64, 2, 16, 16, "f32")
+    assert rng(0, 2, f32, fva.FVA_F32) == fva.FVA_ERR_UNSUPPORTED_SHAPE
+    assert fva.call_raw("fva_sparse_attn_range", ctypes.byref(s), p, p, p, fva.FVA_F16, ctypes.byref(m), p,
+                        ctypes.c_float(0.0), 0, 1, None, None) == fva.FVA_ERR_INVALID_ARG  # o aliases q

@@ -111,3 +111,48 @@ def test_sasa_720p_eight_ranks():
     rank_of = [h * 8 // BH for h in range(BH)]
     budget = [0, 20000, 150000, 0, 80000, 5, 0, 300000]
     _check(wl, C.layer(2), rank_of, budget)
+
+
+@pytest.mark.parametrize("wid_or_wl", [SMALL[0], SMALL[3], 3], ids=lambda w: getattr(w, "name", f"workload{w}"))
+def test_sasa_reads_logits_exported_by_routing(wid_or_wl):
+    """fva_route with mask.logits set exports the block logits (the rows' importance
+    order); they equal the oracle's logits, routing gives the same mask as without the
+    export, and fva_sasa_augment reading them (no pooled Q/K passed) gives the same
+    augmented mask and per-rank counts as recomputing them."""
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import fva
+    if isinstance(wid_or_wl, int):
+        wl, L = synth.WORKLOADS[wid_or_wl], C.layer(wid_or_wl)
+    else:
+        wl, L = wid_or_wl, synth.make_layer(wid_or_wl)
+    BH, nB = wl.B * wl.H, wl.nB
+    rank_of = [h % 2 for h in range(BH)]
+    budget = [5 * nB, 37]
+    run_a, g0a, g1a, added_a = _run_sasa(wl, L, rank_of, budget)
+
+    run = C.GpuRun(wl, L)
+    lay = run.layer
+    lay.mask.logits = torch.full((BH, nB, nB), float("nan"), dtype=torch.float64, device="cuda")
+    lay.route()
+    torch.cuda.synchronize()
+    assert run.status() == 0
+    g0 = run.mask_np()
+    for key in g0:
+        np.testing.assert_array_equal(g0[key], g0a[key])
+    want = _oracle_logits(wl, L, run)
+    got = lay.mask.logits.cpu().numpy()
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+    ws = torch.empty(fva.fva_sasa_workspace_bytes(run.shape), dtype=torch.uint8, device="cuda")
+    rk = torch.tensor(rank_of, dtype=torch.int32, device="cuda")
+    bd = torch.tensor(budget, dtype=torch.int64, device="cuda")
+    added = torch.zeros(len(budget), dtype=torch.int64, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fva.fva_sasa_augment(run.shape, None, None, rk, bd, lay.mask, ws, 2, added, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    np.testing.assert_array_equal(added.cpu().numpy(), added_a)
+    g1 = run.mask_np()
+    for key in g1:
+        np.testing.assert_array_equal(g1[key], g1a[key])
+    # the exported logits are read, not overwritten
+    np.testing.assert_array_equal(lay.mask.logits.cpu().numpy(), got)
