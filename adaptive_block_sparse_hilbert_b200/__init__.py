@@ -5,4 +5,4 @@ The compute path lives in ``libfva.so`` (hand-written sm_100a CUDA behind a C AB
 package does not load the library, so the seeded input generator
 (``adaptive_block_sparse_hilbert_b200.synth``) stays importable on machines without it.
 """
-__all__ = ["fva", "pipeline", "synth"]
+__all__ = ["fva", "migrate", "pipeline", "synth"]

@@ -152,7 +152,13 @@ def measured_sm_imbalance(trace: np.ndarray, sm_count: int):
     finish = np.zeros(sm_count)
     np.maximum.at(finish, sm, (trace[:, 3] - t0).astype(np.float64))
     span = float(trace[:, 3].max() - t0)
+    # launch slots are the work list's positions: the fraction of consecutive slots that
+    # started in list order (within 2 us) shows whether the block scheduler hands out CTAs
+    # in blockIdx order, which the longest-first list relies on
+    st = trace[:, 2].astype(np.int64)
+    in_order = float(np.mean(np.diff(st) >= -2000)) if st.size > 1 else 1.0
     return {"sm_work_max_over_mean": round(float(work.max() / work.mean()), 4),
+            "slots_started_in_list_order": round(in_order, 4),
             "sm_work_max_over_min": round(float(work.max() / max(work.min(), 1.0)), 4),
             "sm_finish_mean_over_span": round(float(finish.mean() / span), 4) if span > 0 else None,
             "span_ms": round(span / 1e6, 3), "ctas": int(trace.shape[0]), "sms": int(sm_count)}
@@ -265,6 +271,67 @@ def sasa_report(layer, s, wl, plan, t_attn_ms: float, kept_blocks: int, dev, str
                     "on the virtual split no rank passes the critical load"}
 
 
+def migration_report(s, wl, q, k, v, o_ref, costs, t_attn_ms: float, head_bytes: float, dev, stream,
+                     ranks: int = 8):
+    """Runtime Load Balancing carried out on `ranks` ranks emulated on this GPU: every rank
+    owns a contiguous slice of the heads, routes them, the loads are gathered, the plan
+    moves heads, their Q, K, V and pooled Q, K are copied into the receivers' own buffers,
+    the donors skip them, the receivers route and attend them and copy O back. The ranks
+    run one after another, so each rank's attention is timed alone on the whole GPU -- what
+    it would take on a GPU of its own. Reported before (no moves) and after, with the
+    outputs checked bit for bit against the unsharded layer's."""
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import migrate
+    if wl.B * wl.H < ranks:
+        return None
+    steps = costs.reshape(wl.B, wl.H, -1).sum(axis=(0, 2)).astype(np.float64)
+    ms_per_step = t_attn_ms / max(float(steps.sum()), 1.0)
+    comm_ms = head_bytes / (PEER_COPY_GBS * 1e9) * 1e3
+    t0 = time.perf_counter()
+    migrate.plan_moves(steps * ms_per_step, ranks, comm_ms, 0.0)
+    sched_ms = (time.perf_counter() - t0) * 1e3
+    objs = [migrate.ShardRank(s, wl.p, wl.k_floor, r, ranks, ms_per_step, device=dev) for r in range(ranks)]
+    sl = [migrate.heads_of_rank(r, ranks, wl.H) for r in range(ranks)]
+    qs = [q[:, :, h.start:h.stop].contiguous() for h in sl]
+    ks = [k[:, :, h.start:h.stop].contiguous() for h in sl]
+    vs = [v[:, :, h.start:h.stop].contiguous() for h in sl]
+    out = {}
+    for label, mig in (("before", False), ("after", True)):
+        os_ = [torch.empty_like(x) for x in qs]
+        marks = []
+
+        def timer(phase, r, fn):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            marks.append((phase, r, e0, e1))
+
+        for rep in range(2):  # the first pass warms up the guests' buffers
+            marks.clear()
+            loads, rank_of, moves = migrate.run_virtual_step(objs, qs, ks, vs, os_, comm_ms, sched_ms,
+                                                             migrate=mig, timer=timer)
+        torch.cuda.synchronize()
+        attn = np.zeros(ranks)
+        for phase, r, e0, e1 in marks:
+            if phase == "attend":
+                attn[r] += e0.elapsed_time(e1)
+        exact = bool(torch.equal(torch.cat(os_, dim=2), o_ref))
+        out[label] = {"attn_ms_per_rank": [round(float(x), 3) for x in attn],
+                      "max_over_mean": round(float(attn.max() / attn.mean()), 4),
+                      "max_over_min": round(float(attn.max() / attn.min()), 4),
+                      "makespan_ms": round(float(attn.max()), 3),
+                      "moves": [[m.head, m.src, m.dst] for m in moves], "outputs_equal_unsharded": exact}
+    status = max(o.dev_status() for o in objs)
+    del objs, qs, ks, vs
+    torch.cuda.empty_cache()
+    return {"ranks": ranks, "heads": wl.H, "comm_ms_per_head": round(comm_ms, 4), "sched_ms": round(sched_ms, 4),
+            "ms_per_tile_step": ms_per_step, **out, "dev_status": status,
+            "note": "ranks emulated one after another on one GPU (each rank's attention timed alone on the GPU); "
+                    "the head transfers are device copies here and NCCL send/recv between GPUs (not measured: "
+                    "one GPU per run)"}
+
+
 def imbalance(costs: np.ndarray, BH: int, n_pairs: int, slots: int):
     out = {}
     ids = np.arange(costs.size)
@@ -283,44 +350,97 @@ def imbalance(costs: np.ndarray, BH: int, n_pairs: int, slots: int):
     return out
 
 
-# ----------------------------------------------------------------------------------- oracle timing
+# ----------------------------------------------------------------------------------- oracle leg
 
-def oracle_sample(wl, L, n_heads: int, rows_per_head: int, seed: int = 0):
-    """Time the float64 oracle on a bounded sample and extrapolate to a full layer (ms)."""
+def oracle_heads(wl, L, perm, heads, rows_per_head: int, seed: int, ambiguity: bool = False, resamples: int = 0):
+    """The float64 oracle over whole heads of one layer (B = 1): reorder + pooling and the
+    full routing of each head, then attention on `rows_per_head` seeded query blocks of it.
+    One record per head: its times in seconds, the query x key token pairs of the sampled
+    rows and of the whole head (the attention work), and with ambiguity=True its CSR mask
+    and the oracle's ambiguity flags, which are computed after the timed part. With
+    resamples = n, n more sets of seeded rows are attended and timed ("resampled": a list of
+    (seconds, pairs) per set) to show the spread of the attention estimate."""
     import oracle as O
+    assert wl.B == 1
     rng = np.random.default_rng(seed)
-    heads = rng.choice(wl.H, size=min(n_heads, wl.H), replace=False)
-    t0 = time.perf_counter()
-    perm, _ = O.hilbert_perm(wl.T, wl.Hg, wl.Wg)
-    t_perm = time.perf_counter() - t0
-    t_reorder = t_route = t_attn = 0.0
-    n_rows = 0
+    nB, N = wl.nB, wl.N
+    sizes = np.minimum(64, N - 64 * np.arange(nB)).astype(np.int64)
+    recs = []
     for h in heads:
         t0 = time.perf_counter()
         q = O.reorder(L.q[:, :, h:h + 1], perm)
         k = O.reorder(L.k[:, :, h:h + 1], perm)
         v = O.reorder(L.v[:, :, h:h + 1], perm)
+        pq, pk = O.block_mean_pool(q), O.block_mean_pool(k)
         t1 = time.perf_counter()
-        R = O.route(O.block_mean_pool(q), O.block_mean_pool(k), wl.d, wl.p, wl.k_floor)
+        R = O.route(pq, pk, wl.d, wl.p, wl.k_floor)
         t2 = time.perf_counter()
-        rows = [(0, 0, int(a)) for a in rng.choice(wl.nB, size=min(rows_per_head, wl.nB), replace=False)]
-        O.block_sparse_attention(q, k, v, R["row_ptr"], R["col_idx"], rows=rows)
+        rows = np.sort(rng.choice(nB, size=min(rows_per_head, nB), replace=False))
+        if rows.size:
+            O.block_sparse_attention(q, k, v, R["row_ptr"], R["col_idx"], rows=[(0, 0, int(a)) for a in rows])
         t3 = time.perf_counter()
-        t_reorder += t1 - t0
-        t_route += t2 - t1
-        t_attn += t3 - t2
-        n_rows += len(rows)
-    nh = len(heads)
-    ms = 1e3 * (t_perm + (t_reorder + t_route) * wl.H / nh + t_attn * (wl.H * wl.nB) / n_rows)
-    if nh == wl.H and n_rows == wl.H * wl.nB:
-        sample = (f"the full layer: reorder, pooling, routing and attention of all {wl.H} heads and all "
-                  f"{wl.nB} query blocks (no extrapolation)")
-    else:
-        sample = (f"{nh} of {wl.H} heads: reorder + pooling + full routing of each sampled head, attention on "
-                  f"{min(rows_per_head, wl.nB)} seeded query blocks per sampled head; time extrapolated linearly "
-                  f"to all heads and all {wl.nB} query blocks (extrapolated)")
-    wall = t_perm + t_reorder + t_route + t_attn
-    return ms, sample, wall
+        rp, ci = R["row_ptr"], R["col_idx"]
+        keys = np.bincount(np.repeat(np.arange(nB), np.diff(rp)), weights=sizes[ci], minlength=nB)
+        pairs = sizes * keys
+        rec = {"head": int(h), "prep_s": t1 - t0, "route_s": t2 - t1, "attn_s": t3 - t2, "rows": int(rows.size),
+               "pairs_sampled": float(pairs[rows].sum()), "pairs_head": float(pairs.sum())}
+        rec["resampled"] = []
+        for _ in range(resamples):
+            rows2 = np.sort(rng.choice(nB, size=min(rows_per_head, nB), replace=False))
+            t4 = time.perf_counter()
+            O.block_sparse_attention(q, k, v, rp, ci, rows=[(0, 0, int(a)) for a in rows2])
+            rec["resampled"].append((time.perf_counter() - t4, float(pairs[rows2].sum())))
+        if ambiguity:
+            Ra = O.route(pq, pk, wl.d, wl.p, wl.k_floor, with_ambiguity=True)
+            rec.update(row_ptr=rp, col_idx=ci, ambiguous=Ra["ambiguous_mass"] | Ra["ambiguous_tie"])
+        recs.append(rec)
+    return recs
+
+
+def oracle_layer_ms(wl, recs, t_perm_s: float) -> float:
+    """One layer's oracle time (ms) from per-head records: reorder, pooling and routing as
+    measured, attention scaled from the sampled rows to the whole head by query x key
+    pairs. Heads without a record count at the mean of the measured heads (a head measured
+    more than once counts at its mean)."""
+    per_head = {}
+    for r in recs:
+        attn = r["attn_s"] * (r["pairs_head"] / r["pairs_sampled"]) if r["pairs_sampled"] > 0 else 0.0
+        per_head.setdefault(r["head"], []).append(r["prep_s"] + r["route_s"] + attn)
+    mean_head = float(np.mean([np.mean(v) for v in per_head.values()]))
+    return 1e3 * (t_perm_s + mean_head * wl.H)
+
+
+def oracle_sample_text(wl, recs) -> str:
+    heads = sorted({r["head"] for r in recs})
+    rows = max(r["rows"] for r in recs)
+    full = rows >= wl.nB and len(heads) == wl.H
+    if full:
+        return (f"the full layer: reorder, pooling, routing and attention of all {wl.H} heads and all "
+                f"{wl.nB} query blocks (no extrapolation)")
+    head_txt = (f"all {wl.H} heads" if len(heads) == wl.H else
+                f"{len(heads)} of {wl.H} heads (the others counted at their mean)")
+    return (f"{head_txt} reordered, pooled and routed in full; attention on {rows} seeded query blocks per "
+            f"head, scaled to the head's kept query x key pairs (extrapolated)")
+
+
+def mask_parity(wl, recs, gpu_row_ptr: np.ndarray, gpu_col_idx: np.ndarray):
+    """Rows of the GPU-routed mask that differ from the oracle's, and how many of them (and
+    of all rows) the oracle flags as ambiguous (a cumulative mass within 1e-6 of p, or
+    logits at the boundary closer than 1e-9 relative). `recs` must cover every head."""
+    nB = wl.nB
+    rows = mism = mism_out = amb = 0
+    for r in sorted(recs, key=lambda x: x["head"]):
+        h = r["head"]
+        orp, oci, a = r["row_ptr"], r["col_idx"], r["ambiguous"]
+        amb += int(a.sum())
+        for i in range(nB):
+            g0, g1 = int(gpu_row_ptr[h * nB + i]), int(gpu_row_ptr[h * nB + i + 1])
+            o0, o1 = int(orp[i]), int(orp[i + 1])
+            if g1 - g0 != o1 - o0 or not np.array_equal(gpu_col_idx[g0:g1], oci[o0:o1]):
+                mism += 1
+                mism_out += int(not a[i])
+        rows += nB
+    return {"rows": rows, "mismatches": mism, "mismatches_outside_band": mism_out, "ambiguous": amb}
 
 
 def cpu_cores():
@@ -341,30 +461,54 @@ def cpu_cores():
 
 # ----------------------------------------------------------------------------------- reference arm
 
+def bench_config(wl, args, world: int) -> dict:
+    """The `config` object of the JSON line; both arms print the same one."""
+    esize = 2 if wl.dtype == "bf16" else 4
+    return {"workload": wl.name, "tokens": wl.N, "grid": [wl.T, wl.Hg, wl.Wg], "heads": wl.H, "head_dim": wl.d,
+            "block": 64, "p": wl.p, "k_floor": wl.k_floor, "order": "head_lpt", "curve": args.curve,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": ("inputs larger than L2" if 3 * wl.B * wl.N * wl.H * wl.d * esize > 126e6 else
+                   "inputs smaller than L2, not flushed") + " (3 x %.1f MB)" % (wl.B * wl.N * wl.H * wl.d * esize / 1e6)}
+
+
 def run_reference(args):
+    """The float64 oracle on the host cores. The K timed steps split the layer's heads
+    between them (every head is reordered, pooled and routed in full exactly once when
+    K <= H); the value is the layer time that the per-head records add up to, with
+    attention scaled from the sampled rows by each head's kept work."""
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
     wl = synth.WORKLOADS[args.workload]
     wl = synth.Workload(**{**wl.__dict__, "p": args.p if args.p is not None else wl.p})
     L = synth.make_layer(wl)
-    vals = []
-    sample = ""
-    for i in range(args.warmup + args.steps):
-        ms, sample, _ = oracle_sample(wl, L, n_heads=args.cpu_heads, rows_per_head=args.cpu_rows, seed=i)
-        if i >= args.warmup:
-            vals.append(ms)
+    import oracle as O
+    t0 = time.perf_counter()
+    perm, _ = (O.rect_curve_perm if args.curve == "rect" else O.hilbert_perm)(wl.T, wl.Hg, wl.Wg)
+    t_perm = time.perf_counter() - t0
+    for w in range(args.warmup):  # one head, one query block each
+        oracle_heads(wl, L, perm, [w % wl.H], 1, seed=10_000 + w)
+    chunks = [c for c in np.array_split(np.arange(wl.H), min(args.steps, wl.H))]
+    recs, walls = [], []
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        recs += oracle_heads(wl, L, perm, chunks[i % len(chunks)], args.cpu_rows, seed=i)
+        walls.append(time.perf_counter() - t0)
     cores, threads = cpu_cores()
-    v = float(np.median(vals))
+    v = oracle_layer_ms(wl, recs, t_perm)
+    sample = oracle_sample_text(wl, recs)
     line = {
         "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "ms/layer", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 3), "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "tokens": wl.N, "heads": wl.H, "head_dim": wl.d, "p": wl.p,
-                   "k_floor": wl.k_floor, "block": 64},
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * float(np.mean(walls)), 3),
+        "extrapolated": "(extrapolated)" in sample,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": bench_config(wl, args, world),
         "cpu_baseline": {"value": round(v, 3), "unit": "ms/layer", "cores": threads, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample + f"; each timed step covers {len(chunks[0])} head(s)",
+                         "affinity_cores": cores},
         "e2e": {"value": round(v, 3), "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": "ms_per_step is the wall time of one timed step (a part of the layer's heads); value is the "
+                "whole layer's oracle time assembled from the per-head records",
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -499,7 +643,7 @@ def run_gpu(args):
         a_idx = np.repeat(np.arange(BH * nB) % nB, np.diff(rp))
         kf = float(4 * d * np.sum(sizes[a_idx] * sizes[ci]))
         costs = layer.mask.tile_cost.cpu().numpy().astype(np.int64)
-        return kept, kf, costs, layer.mask.head_kept.cpu().numpy().astype(np.float64)
+        return kept, kf, costs, layer.mask.head_kept.cpu().numpy().astype(np.float64), rp, ci
 
     per_step = []
     for qq, kk, vv in qkv_steps:
@@ -530,11 +674,21 @@ def run_gpu(args):
                  "mean_head_density_change": round(float(np.mean([x.mean() for x in swings])), 4),
                  "note": "value = reorder + routing + attention + inverse reorder per denoising step, "
                          "each step a fresh layer"}
+        first = (args.warmup) % len(qkv_steps)  # drift step of the first timed iteration
+        by_step = {}
+        for i in range(args.steps):
+            by_step.setdefault((first + i) % len(qkv_steps), []).append(stage[i])
+        drift["per_step_ms"] = [
+            {"step": st_i, "timed": len(v), "layer": round(float(np.mean([x.sum() for x in v])), 3),
+             "route_plus_attn": round(float(np.mean([x[1] + x[2] for x in v])), 3),
+             "route": round(float(np.mean([x[1] for x in v])), 3), "attn": round(float(np.mean([x[2] for x in v])), 3)}
+            for st_i, v in sorted(by_step.items())]
         layer.reorder_inputs(q, k, v)  # step 0 again for the dense and end-to-end runs below
         layer.route()
 
     pk, how = peaks()
     peak_tf = float(pk.get("bf16_tflops_sustained", pk.get("bf16_tflops")))
+    burst_tf = float(pk.get("bf16_tflops", peak_tf))
     hbm = float(pk["hbm_gbs"])
     achieved_tf = kept_flops / (t_attn * 1e-3) / 1e12
     tr = traffic_record(os.path.join(ROOT, "adaptive_block_sparse_hilbert_b200", "csrc", "attn_tc.cu"))
@@ -567,6 +721,32 @@ def run_gpu(args):
     finally:
         fva.fva_set_cta_trace(None)
     sm_measured = measured_sm_imbalance(trace.cpu().numpy(), sm_count)
+
+    # SM-level balance in each work-list order: the slot model, one traced launch and the
+    # attention time (outside the timed region; the layer is routed again in each order)
+    slots_model = imbalance(per_step[0][2], BH, (nB + 1) // 2, 2 * sm_count)
+    by_order = {}
+    for oname, ocode in (("natural", fva.FVA_ORDER_NATURAL), ("lpt", fva.FVA_ORDER_LPT),
+                         ("head_lpt", fva.FVA_ORDER_HEAD_LPT)):
+        layer.order = ocode
+        layer.route()
+        layer.attend()
+        e0, e1 = ev(), ev()
+        e0.record(stream)
+        for _ in range(3):
+            layer.attend()
+        e1.record(stream)
+        fva.fva_set_cta_trace(trace)
+        try:
+            layer.attend()
+            torch.cuda.synchronize()
+        finally:
+            fva.fva_set_cta_trace(None)
+        by_order[oname] = {"attn_ms": round(e0.elapsed_time(e1) / 3, 3), "slots_model": slots_model[oname],
+                           "measured": measured_sm_imbalance(trace.cpu().numpy(), sm_count)}
+    layer.order = fva.FVA_ORDER_HEAD_LPT
+    layer.route()
+    torch.cuda.synchronize()
     del trace
 
     # end to end through the public API with host buffers (pinned), copies inside the timed
@@ -626,14 +806,50 @@ def run_gpu(args):
         for x in per_step:
             r, _ = rlb_report(x[2], BH, (nB + 1) // 2, t_attn, head_bytes)
             rlb["per_step"].append({"before": r["before"], "after": r["after"], "moves": len(r["moves"])})
+    # RLB head migration carried out on 8 ranks emulated on this GPU (step-0 inputs; the
+    # unsharded layer's output on them is the reference)
+    o_ref = torch.empty_like(o)
+    layer.forward(q, k, v, o_ref)
+    migration = None if args.no_migration else migration_report(s, wl, q, k, v, o_ref, costs, t_attn, head_bytes,
+                                                                dev, stream)
+    del o_ref
+    if migration is not None:
+        status = max(status, migration["dev_status"])
     sasa = None if args.no_sasa else sasa_report(layer, s, wl, plan, t_attn, kept, dev, stream)
 
+    # CPU leg (rank 0, one GPU): the float64 oracle timed on the host cores over every head
+    # of the layer, and the oracle's masks compared row by row with the GPU's
     cpu = None
+    parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle as O
         cores, threads = cpu_cores()
-        ms_cpu, sample, wall = oracle_sample(wl, L, n_heads=args.cpu_heads, rows_per_head=args.cpu_rows)
-        cpu = {"value": round(ms_cpu, 1), "unit": "ms/layer", "cores": threads, "kind": "oracle", "sample": sample,
-               "wall_s": round(wall, 1), "affinity_cores": cores}
+        t0 = time.perf_counter()
+        perm_o, _ = (O.rect_curve_perm if args.curve == "rect" else O.hilbert_perm)(wl.T, wl.Hg, wl.Wg)
+        t_perm = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        recs = oracle_heads(wl, L, perm_o, range(wl.H), args.cpu_rows, seed=0, ambiguity=True,
+                            resamples=args.cpu_repeats - 1)
+        wall = time.perf_counter() - t0
+        ms_cpu = oracle_layer_ms(wl, recs, t_perm)
+        # the same heads' attention rows drawn again with other seeds: the spread of the estimate
+        reps = [ms_cpu]
+        for j in range(args.cpu_repeats - 1):
+            again = [{**r, "attn_s": r["resampled"][j][0], "pairs_sampled": r["resampled"][j][1]} for r in recs]
+            reps.append(oracle_layer_ms(wl, again, t_perm))
+        cpu = {"value": round(ms_cpu, 1), "unit": "ms/layer", "cores": threads, "kind": "oracle",
+               "sample": oracle_sample_text(wl, recs), "wall_s": round(wall, 1), "affinity_cores": cores,
+               "repeats_ms": [round(x, 1) for x in reps],
+               "spread": round((max(reps) - min(reps)) / float(np.median(reps)), 4)}
+        parity = mask_parity(wl, recs, per_step[0][4], per_step[0][5])
+        if len(per_step) > 1:
+            parity = {"per_step": [parity]}
+            for st_i in range(1, len(per_step)):
+                rs = oracle_heads(wl, layers_np[st_i], perm_o, range(wl.H), 0, seed=0, ambiguity=True)
+                parity["per_step"].append(mask_parity(wl, rs, per_step[st_i][4], per_step[st_i][5]))
+            for key in ("rows", "mismatches", "mismatches_outside_band", "ambiguous"):
+                parity[key] = int(sum(x[key] for x in parity["per_step"]))
+        parity["against"] = "float64 oracle routing of every row (computed in the CPU leg)"
 
     if rank == 0:
         line = {
@@ -649,12 +865,12 @@ def run_gpu(args):
             "vs_baseline": None,
             "dtype": "bf16" if wl.dtype == "bf16" else "f32",
             "data": "synthetic",
-            "config": {"workload": wl.name, "tokens": N, "grid": [wl.T, wl.Hg, wl.Wg], "heads": wl.H,
-                       "head_dim": d, "block": 64, "p": wl.p, "k_floor": wl.k_floor, "order": "head_lpt", "curve": args.curve,
-                       "parallelism": f"replicas{world}" if world > 1 else "single",
-                       "l2": "inputs larger than L2 (3 x %.0f MB)" % (q.numel() * q.element_size() / 1e6)},
+            "config": bench_config(wl, args, world),
             "kept_tflops": round(achieved_tf, 1),
             "kept_tflops_frac_of_peak": round(achieved_tf / peak_tf, 4),
+            "kept_tflops_frac": {"of_sustained": round(achieved_tf / peak_tf, 4),
+                                 "of_burst": round(achieved_tf / burst_tf, 4),
+                                 "sustained_tflops": peak_tf, "burst_tflops": burst_tf, "source": how},
             "issued_tflops": round(issued_flops / (t_attn * 1e-3) / 1e12, 1),
             "density": round(kept / (BH * nB * nB), 4),
             "stage_ms": {"reorder_qkv": round(t_reorder, 4), "route": round(t_route, 4), "attn": round(t_attn, 4),
@@ -680,7 +896,11 @@ def run_gpu(args):
                          "peak_source": f"{how} bf16_tflops_sustained (kernel timed inside a multi-second loop)"},
             "imbalance_sm_slots": imb,
             "imbalance_sm_measured": sm_measured,
+            "imbalance_by_order": {**by_order, "pages_rank_level": "average rank load imbalance 1.34 -> 1.08 with "
+                                                                   "RLB (Wan2.2 I2V, 8 x H20): whole heads per rank, "
+                                                                   "a much coarser unit than tiles per SM"},
             "rlb_virtual_ranks": rlb,
+            "rlb_migration_virtual_ranks": migration,
             "sasa_virtual_ranks": sasa,
             "e2e": {"value": round(whole_job_ms_per_layer(e2e_ms, world), 3), "unit": "ms/layer",
                     "h2d_bytes_per_step": int(h2d),
@@ -697,6 +917,8 @@ def run_gpu(args):
             line["drift"] = drift
         if cpu is not None:
             line["cpu_baseline"] = cpu
+        if parity is not None:
+            line["mask_parity"] = parity
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -718,10 +940,12 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sasa", action="store_true", help="skip the slack-aware augmentation report")
+    ap.add_argument("--no-migration", action="store_true", help="skip the head-migration report on emulated ranks")
     ap.add_argument("--e2e-groups", type=int, default=None,
                     help="equal head groups of the host-pipelined end-to-end run (default: a ramp 1, 2, 3, 4, ..., 2)")
-    ap.add_argument("--cpu-heads", type=int, default=8)
-    ap.add_argument("--cpu-rows", type=int, default=4)
+    ap.add_argument("--cpu-rows", type=int, default=4, help="query blocks per head the oracle attends")
+    ap.add_argument("--cpu-repeats", type=int, default=3,
+                    help="sets of seeded query blocks the oracle leg attends (their spread is reported)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

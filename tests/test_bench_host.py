@@ -19,6 +19,11 @@ def test_measured_sm_imbalance_hand_trace():
     # span = 500 - 100 = 400 ms; finish = 400, 200, 0 -> mean 200
     assert r["span_ms"] == pytest.approx(400.0)
     assert r["sm_finish_mean_over_span"] == pytest.approx(0.5)
+    # slot 2 started 50 ms after slot 1: both consecutive pairs are in list order
+    assert r["slots_started_in_list_order"] == pytest.approx(1.0)
+    tr2 = tr.copy()
+    tr2[1, 2] = 160 * ms  # slot 1 now starts after slot 2 (150 ms): one of two pairs inverted
+    assert bench.measured_sm_imbalance(tr2, 3)["slots_started_in_list_order"] == pytest.approx(0.5)
 
 
 def test_measured_sm_imbalance_balanced():
@@ -79,3 +84,42 @@ def test_committed_traffic_record_scaling():
     m = r["measured_bytes"]
     assert r["traffic_bytes_per_launch"] == pytest.approx(
         (m["dram__bytes_read.sum"] + m["dram__bytes_write.sum"]) * 75600 / 32760, rel=1e-3)
+
+
+def test_oracle_leg_layer_time_and_mask_parity():
+    """The oracle leg on the tiny workload: every head routed in full; the layer time adds
+    the per-head records; the mask comparison counts exactly the rows that differ."""
+    import oracle as O
+    from adaptive_block_sparse_hilbert_b200 import synth
+    wl = synth.WORKLOADS[0]
+    L = synth.make_layer(wl)
+    perm, _ = O.hilbert_perm(wl.T, wl.Hg, wl.Wg)
+    recs = bench.oracle_heads(wl, L, perm, range(wl.H), wl.nB, seed=0, ambiguity=True, resamples=1)
+    assert [r["head"] for r in recs] == list(range(wl.H))
+    # every row attended: the sampled pairs are the head's pairs, nothing is scaled
+    for r in recs:
+        assert r["pairs_sampled"] == r["pairs_head"] > 0
+        assert len(r["resampled"]) == 1 and r["resampled"][0][1] == r["pairs_head"]
+    ms = bench.oracle_layer_ms(wl, recs, 0.5)
+    want = 1e3 * (0.5 + sum(r["prep_s"] + r["route_s"] + r["attn_s"] for r in recs))
+    assert ms == pytest.approx(want)
+    assert "no extrapolation" in bench.oracle_sample_text(wl, recs)
+    # a head measured twice counts at its mean; missing heads at the mean of the others
+    two = [dict(recs[0], prep_s=1.0, route_s=0.0, attn_s=0.0), dict(recs[0], prep_s=3.0, route_s=0.0, attn_s=0.0)]
+    assert bench.oracle_layer_ms(wl, two, 0.0) == pytest.approx(1e3 * 2.0 * wl.H)
+    # mask parity against the oracle's own CSR: no mismatch
+    R = O.route(O.block_mean_pool(O.reorder(L.q, perm)), O.block_mean_pool(O.reorder(L.k, perm)), wl.d, wl.p,
+                wl.k_floor, with_ambiguity=True)
+    rp, ci = R["row_ptr"].copy(), R["col_idx"].copy()
+    par = bench.mask_parity(wl, recs, rp, ci)
+    assert par == {"rows": wl.H * wl.nB, "mismatches": 0, "mismatches_outside_band": 0,
+                   "ambiguous": int((R["ambiguous_mass"] | R["ambiguous_tie"]).sum())}
+    # drop the last kept block of row 5 (head 0) and change one entry of row 20 (head 1)
+    ci2 = np.delete(ci, rp[6] - 1)
+    rp2 = rp.copy()
+    rp2[6:] -= 1
+    j = rp2[20]
+    ci2[j] = (ci2[j] + 1) % wl.nB if (ci2[j] + 1) % wl.nB not in ci2[rp2[20]:rp2[21]] else ci2[j]
+    changed = int(not np.array_equal(ci2[rp2[20]:rp2[21]], ci[rp[20]:rp[21]]))
+    par = bench.mask_parity(wl, recs, rp2, ci2)
+    assert par["mismatches"] == 1 + changed and par["mismatches_outside_band"] <= par["mismatches"]

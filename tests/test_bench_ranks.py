@@ -63,4 +63,10 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["dtype"] == "f64"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     # default flags sample 4 of the 16 query blocks per head, so the time is extrapolated
-    assert line["cpu_baseline"]["sample"].endswith("(extrapolated)")
+    assert line["extrapolated"] is True and "(extrapolated)" in line["cpu_baseline"]["sample"]
+    assert line["steps"] == 1 and line["ms_per_step"] > 0
+    import bench
+    import argparse
+    from adaptive_block_sparse_hilbert_b200 import synth
+    # the reference arm prints the GPU arm's config object
+    assert line["config"] == bench.bench_config(synth.WORKLOADS[0], argparse.Namespace(curve="hilbert"), 2)
