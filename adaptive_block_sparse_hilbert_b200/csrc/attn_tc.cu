@@ -53,7 +53,11 @@ struct AttnCfg {
   static constexpr int kQBytes = kChunks * kBM * 128;        // 128 rows x 128 B per chunk
   static constexpr int kKVBytes = kChunks * kBN * 128;       // 64 rows x 128 B per chunk
   static constexpr int kSmemData = kQBytes + 2 * kStages * kKVBytes;
-  static constexpr uint32_t kOCol = 128;                     // O columns [128, 128 + D)
+  // S buffers of 64 TMEM columns each, then O: two buffers at d = 128 (2 x 64 + 128 = 256
+  // columns), three at d = 64 (3 x 64 + 64 = 256), so at d = 64 the QK product runs two
+  // steps ahead of P.V and S(j + 3), not S(j + 2), is the one that waits for P(j)
+  static constexpr int kSBufs = (D == 128) ? 2 : 3;
+  static constexpr uint32_t kOCol = kSBufs * 64;             // O columns [kOCol, kOCol + D)
 };
 
 template <int D>
@@ -63,9 +67,12 @@ struct __align__(8) AttnBars {
   uint64_t k_empty[AttnCfg<D>::kStages];
   uint64_t v_full[AttnCfg<D>::kStages];
   uint64_t v_empty[AttnCfg<D>::kStages];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t pv_done;
+  uint64_t s_full[AttnCfg<D>::kSBufs];
+  uint64_t p_full[AttnCfg<D>::kSBufs];
+  // one per S buffer: P.V of step i completes pv_done[i % kSBufs], so a wait for step j - 1
+  // never sees more than one phase of ambiguity (S(j) arriving implies every P.V of a step
+  // <= j - kSBufs is complete)
+  uint64_t pv_done[AttnCfg<D>::kSBufs];
   uint64_t o_full;
   uint64_t drain;
   uint32_t tmem_base;
@@ -130,11 +137,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       mbar_init(&bar.v_full[s], 1);
       mbar_init(&bar.v_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < Cfg::kSBufs; ++i) {
       mbar_init(&bar.s_full[i], 1);
       mbar_init(&bar.p_full[i], 128);
+      mbar_init(&bar.pv_done[i], 1);
     }
-    mbar_init(&bar.pv_done, 1);
     mbar_init(&bar.o_full, 1);
     mbar_init(&bar.drain, 1);
     bar.abort = 0;
@@ -234,10 +241,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       constexpr uint32_t idesc_pv = idesc_f16kind_f32(kBM, D, 0, 1, VF16 ? kFmtF16 : kFmtBF16);
       bool ok = mbar_wait(&bar.q_full, 0, abort_flag, kWaitLimitNs);
       bool issued = false;
+      constexpr int kLag = Cfg::kSBufs - 1;  // P.V of step j - kLag follows the QK of step j
       auto issue_pv = [&](int i) -> bool {
-        const int sb = i & 1;
+        const int sb = i % Cfg::kSBufs;
         const int s = i % Cfg::kStages;
-        if (!mbar_wait(&bar.p_full[sb], (i >> 1) & 1, abort_flag, kWaitLimitNs)) return false;
+        if (!mbar_wait(&bar.p_full[sb], (i / Cfg::kSBufs) & 1, abort_flag, kWaitLimitNs)) return false;
         if (!mbar_wait(&bar.v_full[s], (i / Cfg::kStages) & 1, abort_flag, kWaitLimitNs)) return false;
         tc_fence_after();
         const uint32_t v_base = smem_u32(sV + s * Cfg::kKVBytes);
@@ -247,13 +255,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           mma_ts(tmem + Cfg::kOCol, tmem + sb * 64 + kk * 8, bdesc, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(&bar.v_empty[s]);
-        tc_commit(&bar.pv_done);
+        tc_commit(&bar.pv_done[sb]);
         return true;
       };
       if (ok) tc_fence_after();
       for (int j = 0; j < n_iter && ok; ++j) {
         const int s = j % Cfg::kStages;
-        const int sb = j & 1;
+        const int sb = j % Cfg::kSBufs;
         if (!mbar_wait(&bar.k_full[s], (j / Cfg::kStages) & 1, abort_flag, kWaitLimitNs)) {
           ok = false;
           break;
@@ -272,12 +280,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         issued = true;
         tc_commit(&bar.k_empty[s]);
         tc_commit(&bar.s_full[sb]);
-        if (j >= 1 && !issue_pv(j - 1)) {
+        if (j >= kLag && !issue_pv(j - kLag)) {
           ok = false;
           break;
         }
       }
-      if (ok && n_iter > 0) ok = issue_pv(n_iter - 1);
+      for (int i = n_iter > kLag ? n_iter - kLag : 0; i < n_iter && ok; ++i) ok = issue_pv(i);
       if (ok) {
         tc_commit(&bar.o_full);
       } else {
@@ -303,8 +311,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       const int entry = DENSE ? ((j << 2) | 3) : tile_col[list_base + j];
       const int kb = entry >> 2;
       const bool keep = (entry >> half) & 1;
-      const int sb = j & 1;
-      if (!warp_wait(&bar.s_full[sb], (j >> 1) & 1, abort_flag, kWaitLimitNs)) {
+      const int sb = j % Cfg::kSBufs;
+      if (!warp_wait(&bar.s_full[sb], (j / Cfg::kSBufs) & 1, abort_flag, kWaitLimitNs)) {
         ok = false;
         break;
       }
@@ -337,7 +345,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         if (__any_sync(0xffffffffu, need_o)) {
           // O holds rows rescaled to the old maximum: wait for the PV of step j-1, then
           // O_row *= 2^(m_ref - m_new) for the rows whose maximum moved.
-          if (!warp_wait(&bar.pv_done, (j - 1) & 1, abort_flag, kWaitLimitNs)) {
+          if (!warp_wait(&bar.pv_done[(j - 1) % Cfg::kSBufs], ((j - 1) / Cfg::kSBufs) & 1, abort_flag,
+                         kWaitLimitNs)) {
             ok = false;
             break;
           }
