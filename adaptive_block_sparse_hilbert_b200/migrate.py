@@ -135,25 +135,31 @@ def _flatten(pairs, tensors_of):
 
 
 def run_step(rank_obj, exchange: DistExchange, q, k, v, o, comm_ms: float, sched_ms: float = 0.1,
-             threshold: float = 1.10):
+             threshold: float = 1.10, migrate: bool = True, timer=None):
     """One step of one rank of a process group. q, k, v, o: this rank's raster [B, N, H_r, d]
     slices. comm_ms (P: moving one head) and sched_ms (C: the planner's time) enter the plan,
-    so they must be the same on every rank -- constants, not per-rank measurements. Returns
-    (rank_of, moves); o holds the rank's output when the call returns (its stream ordered
-    after everything the step enqueued)."""
+    so they must be the same on every rank -- constants, not per-rank measurements.
+    migrate=False keeps every head at home (the same collective steps are still taken);
+    `timer`, if given, is called as timer(phase, fn) around the rank's compute phases.
+    Returns (rank_of, moves); o holds the rank's output when the call returns (its stream
+    ordered after everything the step enqueued)."""
     H, R, r = rank_obj.H, exchange.world, exchange.rank
-    rank_obj.prepare(q, k, v)
+    run = timer if timer is not None else (lambda phase, fn: fn())
+    run("prepare", lambda: rank_obj.prepare(q, k, v))
     loads = exchange.all_gather_loads(rank_obj.local_loads(), H, rank_obj.device)
-    rank_of, moves = plan_moves(loads, R, comm_ms, sched_ms, threshold)
+    if migrate:
+        rank_of, moves = plan_moves(loads, R, comm_ms, sched_ms, threshold)
+    else:
+        rank_of, moves = np.array([x for x in range(R) for _ in heads_of_rank(x, R, H)], np.int32), []
     s_in, r_in = transfers(moves, r, "inputs")
     h_in = exchange.transfer(_flatten(s_in, rank_obj.input_tensors), _flatten(r_in, rank_obj.input_buffers))
-    rank_obj.attend_own(skip=[m.head for _, m in s_in])
+    run("attend", lambda: rank_obj.attend_own(skip=[m.head for _, m in s_in]))
     h_in.wait()
-    rank_obj.attend_received([m.head for _, m in r_in])
+    run("attend_received", lambda: rank_obj.attend_received([m.head for _, m in r_in]))
     s_out, r_out = transfers(moves, r, "outputs")
     h_out = exchange.transfer(_flatten(s_out, rank_obj.output_tensors), _flatten(r_out, rank_obj.output_buffers))
     h_out.wait()
-    rank_obj.finish(o)
+    run("finish", lambda: rank_obj.finish(o))
     return rank_of, moves
 
 

@@ -347,6 +347,51 @@ def migration_report(s, wl, q, k, v, o_ref, costs, t_attn_ms: float, head_bytes:
                     "one GPU per run)"}
 
 
+def distributed_migration_report(s, wl, q, k, v, o_ref, costs, t_attn_ms: float, head_bytes: float, dev, dist_mod):
+    """RLB head migration between the GPUs of this process group (one rank per GPU, NCCL):
+    rank r owns heads [r H / R, (r + 1) H / R) of the layer, and one step (route, gather the
+    loads, plan, move heads point to point, attend, return O) runs with and without
+    migration. Reports every rank's step time (CUDA events, max over ranks) and checks
+    every rank's output against the unsharded layer's."""
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import migrate
+    rank, world = dist_mod.get_rank(), dist_mod.get_world_size()
+    if wl.B * wl.H < world:
+        return None
+    steps = costs.reshape(wl.B, wl.H, -1).sum(axis=(0, 2)).astype(np.float64)
+    ms_per_step = t_attn_ms / max(float(steps.sum()), 1.0)
+    comm_ms = (head_bytes + 2.0 * wl.B * wl.nB * wl.d * 8) / (PEER_COPY_GBS * 1e9) * 1e3
+    hs = migrate.heads_of_rank(rank, world, wl.H)
+    obj = migrate.ShardRank(s, wl.p, wl.k_floor, rank, world, ms_per_step, device=dev)
+    qs, ks, vs = (x[:, :, hs.start:hs.stop].contiguous() for x in (q, k, v))
+    ex = migrate.DistExchange()
+    out = {}
+    for label, mig in (("before", False), ("after", True)):
+        o = torch.empty_like(qs)
+        for _ in range(2):  # the first step warms the receivers' buffers up
+            dist_mod.barrier()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            rank_of, moves = migrate.run_step(obj, ex, qs, ks, vs, o, comm_ms, 0.1, migrate=mig)
+            e1.record()
+            torch.cuda.synchronize()
+        t = torch.tensor([e0.elapsed_time(e1), float(torch.equal(o, o_ref[:, :, hs.start:hs.stop]))],
+                         dtype=torch.float64, device=dev)
+        allt = [torch.empty_like(t) for _ in range(world)]
+        dist_mod.all_gather(allt, t)
+        ms = np.array([float(x[0]) for x in allt])
+        out[label] = {"step_ms_per_rank": [round(float(x), 3) for x in ms], "step_ms": round(float(ms.max()), 3),
+                      "max_over_mean": round(float(ms.max() / ms.mean()), 4),
+                      "moves": [[m.head, m.src, m.dst] for m in moves],
+                      "outputs_equal_unsharded": bool(min(float(x[1]) for x in allt) == 1.0)}
+    status = obj.dev_status()
+    del obj, qs, ks, vs
+    return {"ranks": world, "heads": wl.H, "comm_ms_per_head": round(comm_ms, 4), **out, "dev_status": status,
+            "note": "one step per rank: reorder + route of its heads, all-gather of the loads, RLB plan, NCCL "
+                    "send/recv of the migrated heads, attention, O sent back, inverse reorder"}
+
+
 def fp64_gemm_peak_tflops(dev, n: int = 8192, reps: int = 5) -> float:
     """The float64 denominator of the routing GEMM: cuBLAS DGEMM (torch.matmul in float64,
     n x n x n, 2 n^3 FLOP), best of `reps` after a warm-up, CUDA events. A measurement of the
@@ -850,6 +895,11 @@ def run_gpu(args):
     layer.forward(q, k, v, o_ref)
     migration = None if args.no_migration else migration_report(s, wl, q, k, v, o_ref, costs, t_attn, head_bytes,
                                                                 dev, stream)
+    migration_nccl = None
+    if args.migrate and world > 1:
+        migration_nccl = distributed_migration_report(s, wl, q, k, v, o_ref, costs, t_attn, head_bytes, dev, dist)
+        if migration_nccl is not None:
+            status = max(status, migration_nccl["dev_status"])
     del o_ref
     if migration is not None:
         status = max(status, migration["dev_status"])
@@ -943,6 +993,7 @@ def run_gpu(args):
                                                                    "a much coarser unit than tiles per SM"},
             "rlb_virtual_ranks": rlb,
             "rlb_migration_virtual_ranks": migration,
+            "rlb_migration_nccl": migration_nccl,
             "sasa_virtual_ranks": sasa,
             "e2e": {"value": round(whole_job_ms_per_layer(e2e_ms, world), 3), "unit": "ms/layer",
                     "h2d_bytes_per_step": int(h2d),
@@ -983,6 +1034,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sasa", action="store_true", help="skip the slack-aware augmentation report")
     ap.add_argument("--no-migration", action="store_true", help="skip the head-migration report on emulated ranks")
+    ap.add_argument("--migrate", action="store_true",
+                    help="under torchrun with N > 1: also run one head-sharded step with RLB head migration "
+                         "between the GPUs over NCCL and report it (off by default: the replicas line does not "
+                         "depend on it)")
     ap.add_argument("--e2e-groups", type=int, default=None,
                     help="equal head groups of the host-pipelined end-to-end run (default: a ramp 1, 2, 3, 4, ..., 2)")
     ap.add_argument("--cpu-rows", type=int, default=4, help="query blocks per head the oracle attends")

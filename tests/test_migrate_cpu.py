@@ -187,9 +187,17 @@ def _gloo_rank(rank, world, port, out):
         q, k, v = _slices(L, world)[rank]
         o = torch.zeros_like(q)
         obj = OracleRank(WL, rank, world)
-        rank_of, moves = migrate.run_step(obj, migrate.DistExchange(), q, k, v, o, comm_ms=0.0, sched_ms=0.0)
+        phases = []
+        rank_of, moves = migrate.run_step(obj, migrate.DistExchange(), q, k, v, o, comm_ms=0.0, sched_ms=0.0,
+                                          timer=lambda phase, fn: (phases.append(phase), fn()))
         dist.barrier()
-        out[rank] = (o.numpy().copy(), [(m.head, m.src, m.dst) for m in moves], rank_of.tolist())
+        # the same step with every head kept at home: same collective steps, same output
+        o2 = torch.zeros_like(q)
+        _, moves2 = migrate.run_step(OracleRank(WL, rank, world), migrate.DistExchange(), q, k, v, o2, comm_ms=0.0,
+                                     sched_ms=0.0, migrate=False)
+        dist.barrier()
+        out[rank] = (o.numpy().copy(), [(m.head, m.src, m.dst) for m in moves], rank_of.tolist(), phases,
+                     bool(torch.equal(o, o2)), len(moves2))
     finally:
         dist.destroy_process_group()
 
@@ -211,6 +219,8 @@ def test_gloo_ranks_migrate_and_match_the_unsharded_layer():
     for r in range(world):
         hs = migrate.heads_of_rank(r, world, WL.H)
         np.testing.assert_array_equal(res[r][0], want[:, :, hs.start:hs.stop])
+        assert res[r][3] == ["prepare", "attend", "attend_received", "finish"]
+        assert res[r][4] and res[r][5] == 0  # without migration: no moves, the same output
     # the same plan as the in-process emulation
     ranks = [OracleRank(WL, r, world) for r in range(world)]
     parts = _slices(L, world)
