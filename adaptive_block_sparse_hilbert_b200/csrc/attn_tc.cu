@@ -13,18 +13,19 @@
 //   * Warp roles: warp 4 issues TMA tile loads (Q once, then K and V blocks of 64 keys
 //     into a ring of stages), warp 5 issues tcgen05.mma (one thread), warps 0-3 own one
 //     query row per thread (TMEM lane) for the online softmax and the epilogue.
-//   * S = Q K^T (M=128, N=64, K=d, bf16 -> fp32) goes to one of two TMEM buffers; the
-//     softmax warps read it, write P back over it as packed fp16 (bf16 in the bf16-V
-//     variant) and the MMA warp
-//     issues O += P V with P taken straight from TMEM (A operand) and V from shared
+//   * S = Q K^T (M=128, N=64, K=d, bf16 -> fp32) goes to one of two TMEM buffers (three at
+//     d = 64, where the QK product runs two steps ahead of P V); the softmax warps read
+//     it, write P back over it as packed fp16 (bf16 in the bf16-V variant) and the MMA
+//     warp issues O += P V with P taken straight from TMEM (A operand) and V from shared
 //     memory (B operand, MN-major). O stays in TMEM until the epilogue.
 //   * O is rescaled only when a row maximum grows by more than 2^8 (log2 units), so
 //     the exponentials stay <= 256 and the TMEM read-modify-write of O is rare.
 //   * Two CTAs per SM (<= 256 TMEM columns and ~97 KB smem each): while one CTA runs
 //     its softmax, the other keeps the tensor core busy.
-//   * Tiles are launched in the order of the work list (longest first); the hardware
-//     block scheduler hands each free CTA slot the next tile, i.e. greedy list
-//     scheduling.
+//   * CTA i runs the tile at work-list position first_slot + i (longest first); the
+//     hardware block scheduler hands each free CTA slot the next CTA, i.e. greedy list
+//     scheduling, as long as it dispatches in blockIdx order (the per-CTA trace shows
+//     that it does). A work-list entry that names no tile is reported, not followed.
 //   * Every mbarrier wait is bounded (~2 s); on expiry the CTA reports
 //     FVA_DEVERR_TIMEOUT, drains its own TMA loads and MMAs, frees TMEM and exits.
 #include <math.h>

@@ -209,3 +209,67 @@ def test_dense_full_size_sampled_480p():
         gv = o[0, bh, torch.as_tensor(rows, device="cuda")].float().cpu().numpy()
         mx, mean = C.err_stats(gv, want)
         assert mx <= C.BF16_MAX_ABS and mean <= C.BF16_MEAN_ABS, (mx, mean)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_sparse_attn_range_slices_the_work_list(d):
+    """fva_sparse_attn_range: two ranges that cover the work list give fva_sparse_attn's
+    output bit for bit; a range leaves the rows of every tile outside it untouched."""
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import fva
+    wl = synth.custom_workload(3, 12, 17, 3, d, "bf16", seed=46)   # nB = 10, 15 pair tiles
+    run = C.GpuRun(wl, synth.make_layer(wl))
+    lay = run.layer
+    lay.attend()
+    torch.cuda.synchronize()
+    full = lay.oh.clone()
+    tiles = fva.fva_num_tiles(run.shape)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o = torch.full_like(full, float("nan"))
+    for first, n in ((0, 6), (6, tiles - 6)):
+        fva.fva_sparse_attn_range(run.shape, lay.qh, lay.kh, lay.vh, lay.mask, o, first, n, 0.0, st)
+    fva.fva_sparse_attn_range(run.shape, lay.qh, lay.kh, lay.vh, lay.mask, o, 3, 0, 0.0, st)  # empty: no launch
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(o, full)
+    # only the first 6 slots: their tiles' rows are written, every other row keeps its NaN
+    o = torch.full_like(full, float("nan"))
+    fva.fva_sparse_attn_range(run.shape, lay.qh, lay.kh, lay.vh, lay.mask, o, 0, 6, 0.0, st)
+    torch.cuda.synchronize()
+    wlist = lay.mask.worklist.cpu().numpy()
+    n_pairs = (wl.nB + 1) // 2
+    written = torch.zeros(wl.H, wl.N, dtype=torch.bool)
+    for tile in wlist[:6]:
+        h, t = divmod(int(tile), n_pairs)
+        written[h, t * 128:min(t * 128 + 128, wl.N)] = True
+    got = o[0].cpu()
+    assert torch.equal(got[written], full[0].cpu()[written])
+    assert torch.isnan(got[~written].float()).all()
+
+
+def test_work_list_entry_out_of_range_is_reported_not_followed():
+    """A work-list entry that names no tile: the kernel reports FVA_DEVERR_BAD_LIST, its CTA
+    writes nothing, and every other tile's rows are still computed."""
+    import torch
+    from adaptive_block_sparse_hilbert_b200 import fva
+    wl = synth.custom_workload(3, 12, 17, 2, 128, "bf16", seed=47)   # nB = 10, 10 pair tiles
+    run = C.GpuRun(wl, synth.make_layer(wl))
+    lay = run.layer
+    lay.attend()
+    torch.cuda.synchronize()
+    full = lay.oh.clone()
+    bad_slot = 4
+    victim = int(lay.mask.worklist[bad_slot].item())
+    lay.mask.worklist[bad_slot] = fva.fva_num_tiles(run.shape) + 7   # no such tile
+    o = torch.full_like(full, float("nan"))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fva.fva_sparse_attn(run.shape, lay.qh, lay.kh, lay.vh, lay.mask, o, 0.0, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == fva.FVA_DEVERR_BAD_LIST
+    n_pairs = (wl.nB + 1) // 2
+    h, t = divmod(victim, n_pairs)
+    skipped = torch.zeros(wl.H, wl.N, dtype=torch.bool)
+    skipped[h, t * 128:min(t * 128 + 128, wl.N)] = True
+    got = o[0].cpu()
+    assert torch.isnan(got[skipped].float()).all()                  # the named-nothing CTA wrote nothing
+    assert torch.equal(got[~skipped], full[0].cpu()[~skipped])     # the rest is intact
