@@ -228,3 +228,50 @@ def test_gloo_ranks_migrate_and_match_the_unsharded_layer():
     _, _, vmoves = migrate.run_virtual_step(ranks, [p[0] for p in parts], [p[1] for p in parts],
                                             [p[2] for p in parts], outs, comm_ms=0.0)
     assert [(m.head, m.src, m.dst) for m in vmoves] == [tuple(x) for x in moves]
+
+
+class _DyingDonor(OracleRank):
+    """A rank that fails on the host after the plan, before it sends its migrated head."""
+
+    def input_tensors(self, m):
+        raise RuntimeError("donor failed before sending")
+
+
+def _gloo_failing_rank(rank, world, port, out):
+    import datetime
+    import time
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=3))
+    L = synth.make_layer(WL)
+    q, k, v = _slices(L, world)[rank]
+    o = torch.zeros_like(q)
+    obj = (_DyingDonor if rank == 0 else OracleRank)(WL, rank, world)
+    t0 = time.time()
+    try:
+        migrate.run_step(obj, migrate.DistExchange(), q, k, v, o, comm_ms=0.0, sched_ms=0.0)
+        out[rank] = ("finished", time.time() - t0, "")
+    except Exception as e:  # noqa: BLE001 -- the outcome is what the test checks
+        out[rank] = (type(e).__name__, time.time() - t0, str(e)[:200])
+    if rank == 0:
+        time.sleep(6.0)  # the failed rank stays up but silent, so the others' waits must time out
+    # no barrier or destroy: rank 0 is gone as far as the others are concerned
+
+
+def test_gloo_rank_failing_mid_step_ends_the_receivers_wait():
+    """A donor that fails after the plan never sends its head and stays silent; the
+    receiver's wait for it ends with the process group's timeout (3 s here) as an error, not
+    a hang, and a rank with no transfer finishes its own heads."""
+    import torch.multiprocessing as mp
+    world = 3
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_gloo_failing_rank, args=(world, port, out), nprocs=world, start_method="spawn",
+                           join=True)
+        res = dict(out)
+    # the plan of this layer moves head 0 from rank 0 to rank 2 and head 4 from rank 2 to 0
+    assert res[0][0] == "RuntimeError" and "donor failed" in res[0][2]
+    assert res[2][0] == "RuntimeError" and 2.5 < res[2][1] < 30.0, res[2]
+    assert "Timed out" in res[2][2], res[2]
+    assert res[1][0] == "finished", res[1]
