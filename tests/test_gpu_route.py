@@ -175,3 +175,16 @@ def test_route_full_size_rect_curve(wid):
     """The same acceptance with tokens ordered by the generalized (rectangular) Hilbert curve."""
     wl = synth.WORKLOADS[wid]
     _check_route(wl, C.layer(wid), wl.p, wl.k_floor, order=2, curve=1)
+
+
+@pytest.mark.parametrize("wid", [1, 3])
+def test_rect_curve_layer_attends_within_tolerance(wid):
+    """The generalized-curve token order end to end: masks against the oracle routed on the
+    same order, then sampled attention rows (densest, sparsest, tail, seeded) against the
+    oracle's attention on that order."""
+    wl = synth.WORKLOADS[wid]
+    L = C.layer(wid)
+    run, g, _ = _check_route(wl, L, wl.p, wl.k_floor, order=2, curve=1)
+    mx, mean, n_rows = C.sampled_attention_errors(run, wl, L, g, 3, seed=60 + wid, curve=1)
+    print(f"{wl.name} (generalized curve): sampled {n_rows} query blocks max-abs {mx:.3e} mean-abs {mean:.3e}")
+    assert mx <= C.BF16_MAX_ABS and mean <= C.BF16_MEAN_ABS
