@@ -263,7 +263,9 @@ FVA_API int fva_build_tiles(const fva_shape* s, const fva_mask* mask, int order,
  *     v_dtype == FVA_BF16: P is rounded to bf16 for P.V.
  *   s->dtype == FVA_F32 (CUDA cores, d in {32, 64, 128}): v_dtype must be FVA_F32.
  * scale <= 0 selects 1/sqrt(d). Reads mask->tile_ptr, tile_col, worklist (bf16) or
- * mask->row_ptr, col_idx (fp32). o must not overlap q, k or v.
+ * mask->row_ptr, col_idx (fp32). o must not overlap q, k or v. A work-list entry that names
+ * no tile, or a tile-list entry naming a key block out of range, sets FVA_DEVERR_BAD_LIST in
+ * dev_status; that CTA writes no output rows (bf16 path).
  * A row that keeps no key block (possible only in a caller-made mask: fva_route keeps at
  * least one block per row) has an empty softmax; its output rows are written as zeros.
  */
