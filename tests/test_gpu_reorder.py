@@ -86,6 +86,12 @@ SMALL = [
     synth.custom_workload(2, 5, 7, 2, 64, "f32", seed=14),       # N = 70
     synth.custom_workload(3, 12, 17, 3, 128, "bf16", seed=15, B=2),  # two batch entries
     synth.custom_workload(3, 5, 7, 2, 64, "f32", seed=16, B=3),     # three entries, fp32
+    # rows shorter than 256 B move two or four adjacent heads per CTA
+    synth.custom_workload(3, 10, 13, 4, 32, "bf16", seed=17),           # 64 B rows, 4 heads per CTA
+    synth.custom_workload(3, 10, 13, 6, 32, "bf16", seed=18),           # 64 B rows, H = 6: 2 per CTA
+    synth.custom_workload(2, 9, 11, 2, 64, "bf16", seed=19, B=2),       # 128 B rows, 2 per CTA, B = 2
+    synth.custom_workload(2, 9, 11, 4, 32, "f32", seed=20),             # 128 B rows, 2 per CTA
+    synth.custom_workload(3, 7, 9, 4, 16, "f32", seed=21),              # 64 B rows, 4 per CTA, N = 189
 ]
 
 
