@@ -24,10 +24,9 @@ namespace fva {
 // ---------------------------------------------------------------------------------
 // Block logits
 // ---------------------------------------------------------------------------------
-constexpr int kST = 128;  // output tile (rows and columns)
-
-constexpr int kDK = 16;       // d-chunk staged per step (every supported d is a multiple of 16)
+constexpr int kDK = 16;       // d-chunk per pipeline stage (every supported d is a multiple of 16)
 constexpr int kDP = kDK + 4;  // padded row (doubles): a half-warp's fragment loads hit 32 banks
+constexpr int kStages = 3;    // d-chunks in flight, so one barrier per chunk suffices
 
 __device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, double b) {
   asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
@@ -35,81 +34,102 @@ __device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, dou
                : "d"(a), "d"(b));
 }
 
-// grid: (ceil(nB/128), ceil(nB/128), B*H); 8 warps as 2 (rows) x 4 (columns), each a
-// 64 x 32 block of logits in 8 x 4 MMA tiles of 8 x 8 (lane (g, t) holds A[g][t], B[t][g]
-// and C[g][2t], C[g][2t+1] of a tile).
-__global__ void __launch_bounds__(256, 1) route_scores_kernel(const double* __restrict__ pq,
-                                                              const double* __restrict__ pk,
-                                                              double* __restrict__ S, int nB, int d,
-                                                              double sqrt_d) {
-  __shared__ __align__(16) double As[kST][kDP];
-  __shared__ __align__(16) double Bs[kST][kDP];
+// 16-byte global -> shared copy; with `valid` false the destination is zero-filled and
+// nothing is read
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all_but_one() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
+// A warp computes MI x NI MMA tiles of 8 x 8 (lane (g, t) holds A[g][t], B[t][g] and
+// C[g][2t], C[g][2t+1] of a tile); a CTA is WR x WC warps.
+template <int MI, int NI, int WR, int WC>
+struct ScoresCfg {
+  static constexpr int kMI = MI, kNI = NI, kWR = WR, kWC = WC;
+  static constexpr int kBM = 8 * MI * WR;            // CTA tile rows (query blocks)
+  static constexpr int kBN = 8 * NI * WC;            // CTA tile columns (key blocks)
+  static constexpr int kThreads = 32 * WR * WC;
+  static constexpr int kStageD = (kBM + kBN) * kDP;  // doubles per stage
+  static constexpr size_t kSmem = static_cast<size_t>(kStages) * kStageD * 8;
+};
+// 128 x 64 logits per CTA as 4 x 2 warps of 32 x 32, two CTAs per SM: sixteen warps hide
+// the MMA and shared-memory latencies, and one CTA's epilogue overlaps the other's products.
+using Scores = ScoresCfg<4, 4, 4, 2>;
+constexpr int kScoresCtasPerSm = 2;
+
+// grid: (ceil(nB / kBN), ceil(nB / kBM), B*H). Every logit is the sum over d in ascending
+// order, four products per MMA step, divided by sqrt(d) at the end; the tiling changes no
+// bit of it.
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, kScoresCtasPerSm)
+    route_scores_kernel(const double* __restrict__ pq, const double* __restrict__ pk, double* __restrict__ S,
+                        int nB, int d, double sqrt_d) {
+  constexpr int MI = C::kMI, NI = C::kNI, BM = C::kBM, BN = C::kBN;
+  extern __shared__ __align__(16) double sm_d[];
   const int bh = blockIdx.z;
-  const int a0 = blockIdx.y * kST, b0 = blockIdx.x * kST;
+  const int a0 = blockIdx.y * BM, b0 = blockIdx.x * BN;
   const double* Q = pq + static_cast<int64_t>(bh) * nB * d;
   const double* K = pk + static_cast<int64_t>(bh) * nB * d;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wm = warp & 1, wn = warp >> 1;
+  const int wm = warp % C::kWR, wn = warp / C::kWR;
   const int g = lane >> 2, t = lane & 3;
-  double acc[8][4][2];
+  double acc[MI][NI][2];
 #pragma unroll
-  for (int mi = 0; mi < 8; ++mi)
+  for (int mi = 0; mi < MI; ++mi)
 #pragma unroll
-    for (int ni = 0; ni < 4; ++ni) acc[mi][ni][0] = acc[mi][ni][1] = 0.0;
+    for (int ni = 0; ni < NI; ++ni) acc[mi][ni][0] = acc[mi][ni][1] = 0.0;
 
-  // each thread stages eight consecutive d-elements of one row of each tile
-  const int lr = threadIdx.x >> 1;
-  const int lc = (threadIdx.x & 1) * 8;
-  const int ga = a0 + lr, gb = b0 + lr;
-  double2 qv[4], kv[4];
-  auto fetch = [&](int i0) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      qv[j] = make_double2(0.0, 0.0);
-      kv[j] = qv[j];
-    }
-    if (ga < nB) {
-      const double2* src = reinterpret_cast<const double2*>(Q + static_cast<int64_t>(ga) * d + i0 + lc);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) qv[j] = src[j];
-    }
-    if (gb < nB) {
-      const double2* src = reinterpret_cast<const double2*>(K + static_cast<int64_t>(gb) * d + i0 + lc);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) kv[j] = src[j];
+  // stage rows: BM rows of pooled Q, then BN rows of pooled K, 8 x 16 bytes each
+  auto issue = [&](int chunk) {
+    double* st = sm_d + (chunk % kStages) * C::kStageD;
+    const int i0 = chunk * kDK;
+    for (int c = threadIdx.x; c < (BM + BN) * 8; c += C::kThreads) {
+      const int r = c >> 3, part = c & 7;
+      const bool is_q = r < BM;
+      const int gr = is_q ? a0 + r : b0 + (r - BM);
+      const bool ok = gr < nB;
+      const double* src = (is_q ? Q : K) + static_cast<int64_t>(ok ? gr : 0) * d + i0 + 2 * part;
+      cp_async16(st + r * kDP + 2 * part, src, ok);
     }
   };
-  fetch(0);
-  for (int i0 = 0; i0 < d; i0 += kDK) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      *reinterpret_cast<double2*>(&As[lr][lc + 2 * j]) = qv[j];
-      *reinterpret_cast<double2*>(&Bs[lr][lc + 2 * j]) = kv[j];
-    }
-    __syncthreads();
-    if (i0 + kDK < d) fetch(i0 + kDK);
+  const int nk = d / kDK;
+  issue(0);
+  cp_async_commit();
+  if (nk > 1) issue(1);
+  cp_async_commit();
+  for (int c = 0; c < nk; ++c) {
+    cp_async_wait_all_but_one();  // this thread's copies of chunk c have landed
+    __syncthreads();              // everyone's have, and chunk c - 1 is no longer read
+    if (c + 2 < nk) issue(c + 2);
+    cp_async_commit();
+    const double* As = sm_d + (c % kStages) * C::kStageD;
+    const double* Bs = As + BM * kDP;
 #pragma unroll
     for (int kk = 0; kk < kDK; kk += 4) {
-      double af[8], bf[4];
+      double af[MI], bf[NI];
 #pragma unroll
-      for (int mi = 0; mi < 8; ++mi) af[mi] = As[wm * 64 + mi * 8 + g][kk + t];
+      for (int mi = 0; mi < MI; ++mi) af[mi] = As[(wm * 8 * MI + mi * 8 + g) * kDP + kk + t];
 #pragma unroll
-      for (int ni = 0; ni < 4; ++ni) bf[ni] = Bs[wn * 32 + ni * 8 + g][kk + t];
+      for (int ni = 0; ni < NI; ++ni) bf[ni] = Bs[(wn * 8 * NI + ni * 8 + g) * kDP + kk + t];
 #pragma unroll
-      for (int mi = 0; mi < 8; ++mi)
+      for (int mi = 0; mi < MI; ++mi)
 #pragma unroll
-        for (int ni = 0; ni < 4; ++ni) dmma_8x8x4(acc[mi][ni][0], acc[mi][ni][1], af[mi], bf[ni]);
+        for (int ni = 0; ni < NI; ++ni) dmma_8x8x4(acc[mi][ni][0], acc[mi][ni][1], af[mi], bf[ni]);
     }
-    __syncthreads();
   }
 #pragma unroll
-  for (int mi = 0; mi < 8; ++mi) {
-    const int a = a0 + wm * 64 + mi * 8 + g;
+  for (int mi = 0; mi < MI; ++mi) {
+    const int a = a0 + wm * 8 * MI + mi * 8 + g;
     if (a >= nB) continue;
     double* dst = S + (static_cast<int64_t>(bh) * nB + a) * nB;
 #pragma unroll
-    for (int ni = 0; ni < 4; ++ni) {
-      const int b = b0 + wn * 32 + ni * 8 + 2 * t;
+    for (int ni = 0; ni < NI; ++ni) {
+      const int b = b0 + wn * 8 * NI + ni * 8 + 2 * t;
       if (b < nB) dst[b] = acc[mi][ni][0] / sqrt_d;
       if (b + 1 < nB) dst[b + 1] = acc[mi][ni][1] / sqrt_d;
     }
@@ -446,36 +466,63 @@ __global__ void route_select_kernel(const double* __restrict__ S, int nB, int nW
 // ---------------------------------------------------------------------------------
 // Scans, per-head counts
 // ---------------------------------------------------------------------------------
-// Exclusive scan of n int32 into out[0..n] by one 1024-thread block; returns total.
+// Exclusive scan of n int32 into out[0..n] by one 1024-thread block; returns the total.
+// The block walks the array in chunks of 4 x blockDim.x consecutive elements (each thread
+// four neighbours, so loads and stores are coalesced), loading the next chunk before it
+// combines the current one; `smem` holds 33 int64.
 __device__ int64_t block_exclusive_scan(const int32_t* __restrict__ in, int32_t* __restrict__ out,
-                                        int64_t n, int64_t* smem_warp /*[32]*/) {
+                                        int64_t n, int64_t* smem) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t chunk = (n + blockDim.x - 1) / blockDim.x;
-  const int64_t lo = tid * chunk;
-  const int64_t hi = lo + chunk < n ? lo + chunk : n;
-  int64_t local = 0;
-  for (int64_t i = lo; i < hi; ++i) local += in[i];
-  int64_t inc = local;
+  const int64_t chunk = 4 * static_cast<int64_t>(blockDim.x);
+  auto load = [&](int64_t base, int32_t* v) {
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int64_t v = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += v;
+    for (int q = 0; q < 4; ++q) {
+      const int64_t i = base + 4 * tid + q;
+      v[q] = i < n ? in[i] : 0;
+    }
+  };
+  int32_t cur[4], nxt[4];
+  load(0, cur);
+  int64_t run = 0;  // sum of every chunk before this one
+  for (int64_t base = 0; base < n; base += chunk) {
+    if (base + chunk < n) load(base + chunk, nxt);
+    const int64_t local = static_cast<int64_t>(cur[0]) + cur[1] + cur[2] + cur[3];
+    int64_t inc = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t t = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += t;
+    }
+    if (lane == 31) smem[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {  // scan of the warp totals
+      const int nw = static_cast<int>(blockDim.x >> 5);
+      const int64_t wv = lane < nw ? smem[lane] : 0;
+      int64_t wi = wv;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int64_t t = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += t;
+      }
+      if (lane < nw) smem[lane] = wi - wv;
+      if (lane == 31) smem[32] = wi;
+    }
+    __syncthreads();
+    int64_t x = run + smem[warp] + inc - local;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int64_t i = base + 4 * tid + q;
+      if (i < n) out[i] = static_cast<int32_t>(x);
+      x += cur[q];
+    }
+    run += smem[32];
+    __syncthreads();  // smem is rewritten by the next chunk
+#pragma unroll
+    for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
   }
-  if (lane == 31) smem_warp[warp] = inc;
+  if (tid == 0) out[n] = static_cast<int32_t>(run);
   __syncthreads();
-  int64_t warp_base = 0, total = 0;
-  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
-    if (w < warp) warp_base += smem_warp[w];
-    total += smem_warp[w];
-  }
-  int64_t run = warp_base + inc - local;
-  for (int64_t i = lo; i < hi; ++i) {
-    out[i] = static_cast<int32_t>(run);
-    run += in[i];
-  }
-  if (tid == 0) out[n] = static_cast<int32_t>(total);
-  __syncthreads();
-  return total;
+  return run;
 }
 
 __global__ void __launch_bounds__(1024) finish_kernel(const int32_t* __restrict__ row_cnt, int64_t rows,
@@ -484,7 +531,7 @@ __global__ void __launch_bounds__(1024) finish_kernel(const int32_t* __restrict_
                                                       int32_t* tile_ptr, int64_t* head_kept, int64_t* head_load,
                                                       int64_t capacity, int64_t tile_capacity,
                                                       int32_t* dev_status) {
-  __shared__ int64_t sw[32];
+  __shared__ int64_t sw[33];
   int64_t total_rows = -1;
   if (row_cnt) total_rows = block_exclusive_scan(row_cnt, row_ptr, rows, sw);
   const int64_t total_tiles = block_exclusive_scan(tile_cost, tile_ptr, tiles, sw);
@@ -720,8 +767,13 @@ cudaError_t launch_route(const Dims& D, const double* pq, const double* pk, doub
 
 cudaError_t launch_route_scores(const Dims& D, const double* pq, const double* pk, double* scores, cudaStream_t st) {
   const int nB = static_cast<int>(D.nB);
-  const dim3 grid((nB + kST - 1) / kST, (nB + kST - 1) / kST, static_cast<unsigned>(D.BH));
-  route_scores_kernel<<<grid, 256, 0, st>>>(pq, pk, scores, nB, static_cast<int>(D.d), sqrt(static_cast<double>(D.d)));
+  const dim3 grid((nB + Scores::kBN - 1) / Scores::kBN, (nB + Scores::kBM - 1) / Scores::kBM,
+                  static_cast<unsigned>(D.BH));
+  cudaError_t e = cudaFuncSetAttribute(route_scores_kernel<Scores>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(Scores::kSmem));
+  if (e != cudaSuccess) return e;
+  route_scores_kernel<Scores><<<grid, Scores::kThreads, Scores::kSmem, st>>>(pq, pk, scores, nB, static_cast<int>(D.d),
+                                                                             sqrt(static_cast<double>(D.d)));
   return cudaGetLastError();
 }
 

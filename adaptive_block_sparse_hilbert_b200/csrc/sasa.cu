@@ -14,7 +14,11 @@
 //      skipped entry, a 64-bit key that orders like P (the bits of the positive double P,
 //      plus one; kept entries get 0);
 //   2. an exact radix select fixes, 8 bits per pass from the top, the key tau_r of each
-//      rank's budget-th largest entry (per-CTA shared histograms, one picking step per pass);
+//      rank's budget-th largest entry (per-CTA shared histograms, one picking step per pass).
+//      Once two digits are fixed, the entries that still match their rank's prefix are
+//      copied into a compact list (key and row), and the remaining six passes and the tie
+//      count read that list instead of every entry; when the list would not fit its
+//      capacity they read every entry, with the same result;
 //   3. entries equal to tau_r are shared out in (head, query block) order, lower key block
 //      first within a row, to fill the budget exactly;
 //   4. the new kept bitmask is old | key > tau_r | the allotted ties, and the tile lists,
@@ -85,16 +89,21 @@ __global__ void sasa_init_kernel(const int64_t* __restrict__ budget, int R, cons
   if (added) added[r] = b < t ? b : t;
 }
 
-// histogram of the next 8-bit digit of the keys that match their rank's prefix
-__global__ void __launch_bounds__(512) sasa_hist_kernel(const uint64_t* __restrict__ keys, int64_t rows, int nB,
-                                                        const int32_t* __restrict__ rank_of, int R,
-                                                        const unsigned long long* __restrict__ prefix,
-                                                        const unsigned long long* __restrict__ pmask,
-                                                        const long long* __restrict__ need, int shift,
-                                                        unsigned* hist) {
-  extern __shared__ unsigned sh[];
-  for (int i = threadIdx.x; i < R * kSasaBins; i += blockDim.x) sh[i] = 0u;
-  __syncthreads();
+// The entries (key, row) of selecting ranks that match their rank's prefix after two
+// digits. `count` keeps counting past `capacity`, so a list that did not fit is known.
+struct CompactList {
+  uint64_t* keys;
+  int64_t* rows;
+  unsigned long long* count;
+  unsigned long long capacity;
+  __device__ bool holds_all() const { return count != nullptr && *count <= capacity; }
+};
+
+__global__ void __launch_bounds__(512) sasa_compact_kernel(const uint64_t* __restrict__ keys, int64_t rows, int nB,
+                                                           const int32_t* __restrict__ rank_of, int R,
+                                                           const unsigned long long* __restrict__ prefix,
+                                                           const unsigned long long* __restrict__ pmask,
+                                                           const long long* __restrict__ need, CompactList cl) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
@@ -102,9 +111,56 @@ __global__ void __launch_bounds__(512) sasa_hist_kernel(const uint64_t* __restri
     if (rk < 0 || need[rk] <= 0) continue;
     const uint64_t pf = prefix[rk], pm = pmask[rk];
     const uint64_t* k = keys + r * nB;
-    for (int b = lane; b < nB; b += 32) {
-      const uint64_t v = k[b];
-      if (v != 0 && (v & pm) == pf) atomicAdd(&sh[rk * kSasaBins + static_cast<int>((v >> shift) & 255u)], 1u);
+    for (int b0 = 0; b0 < nB; b0 += 32) {
+      const int b = b0 + lane;
+      const uint64_t v = b < nB ? k[b] : 0ull;
+      const bool in = v != 0 && (v & pm) == pf;
+      const unsigned m = __ballot_sync(0xffffffffu, in);
+      if (m == 0) continue;
+      unsigned long long base = 0;
+      if (lane == 0) base = atomicAdd(cl.count, static_cast<unsigned long long>(__popc(m)));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      const unsigned long long j = base + __popc(m & ((1u << lane) - 1u));
+      if (in && j < cl.capacity) {
+        cl.keys[j] = v;
+        cl.rows[j] = r;
+      }
+    }
+  }
+}
+
+// histogram of the next 8-bit digit of the keys that match their rank's prefix
+// (reads the compact list instead of every entry when `cl` is given and holds them all)
+__global__ void __launch_bounds__(512) sasa_hist_kernel(const uint64_t* __restrict__ keys, int64_t rows, int nB,
+                                                        const int32_t* __restrict__ rank_of, int R,
+                                                        const unsigned long long* __restrict__ prefix,
+                                                        const unsigned long long* __restrict__ pmask,
+                                                        const long long* __restrict__ need, int shift,
+                                                        unsigned* hist, CompactList cl) {
+  extern __shared__ unsigned sh[];
+  for (int i = threadIdx.x; i < R * kSasaBins; i += blockDim.x) sh[i] = 0u;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  if (cl.holds_all()) {
+    const int64_t n = static_cast<int64_t>(*cl.count);
+    for (int64_t j = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; j < n;
+         j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      const uint64_t v = cl.keys[j];
+      const int rk = rank_of_row(rank_of, cl.rows[j], nB, R);
+      if (rk >= 0 && need[rk] > 0 && (v & pmask[rk]) == prefix[rk])
+        atomicAdd(&sh[rk * kSasaBins + static_cast<int>((v >> shift) & 255u)], 1u);
+    }
+  } else {
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+      const int rk = rank_of_row(rank_of, r, nB, R);
+      if (rk < 0 || need[rk] <= 0) continue;
+      const uint64_t pf = prefix[rk], pm = pmask[rk];
+      const uint64_t* k = keys + r * nB;
+      for (int b = lane; b < nB; b += 32) {
+        const uint64_t v = k[b];
+        if (v != 0 && (v & pm) == pf) atomicAdd(&sh[rk * kSasaBins + static_cast<int>((v >> shift) & 255u)], 1u);
+      }
     }
   }
   __syncthreads();
@@ -138,13 +194,16 @@ __global__ void sasa_pick_kernel(unsigned* hist, int R, int shift, unsigned long
 }
 
 // entries equal to tau_r per row (tie candidates)
+// (every entry is read only when the compact list does not hold them all; tie_take starts
+// at zero)
 __global__ void __launch_bounds__(256) sasa_ties_count_kernel(const uint64_t* __restrict__ keys, int64_t rows,
                                                               int nB, const int32_t* __restrict__ rank_of, int R,
                                                               const unsigned long long* __restrict__ prefix,
-                                                              const long long* __restrict__ need, int32_t* tie_take) {
+                                                              const long long* __restrict__ need, int32_t* tie_take,
+                                                              CompactList cl) {
   const int lane = threadIdx.x & 31;
   const int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (r >= rows) return;
+  if (r >= rows || cl.holds_all()) return;
   const int rk = rank_of_row(rank_of, r, nB, R);
   int n = 0;
   if (rk >= 0 && need[rk] > 0) {
@@ -154,6 +213,22 @@ __global__ void __launch_bounds__(256) sasa_ties_count_kernel(const uint64_t* __
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
   if (lane == 0) tie_take[r] = n;
+}
+
+// the same counts from the compact list, when it holds every candidate (ties match the
+// prefix, so all of them are in it)
+__global__ void __launch_bounds__(512) sasa_ties_compact_kernel(int nB, const int32_t* __restrict__ rank_of, int R,
+                                                                const unsigned long long* __restrict__ prefix,
+                                                                const long long* __restrict__ need, int32_t* tie_take,
+                                                                CompactList cl) {
+  if (!cl.holds_all()) return;
+  const int64_t n = static_cast<int64_t>(*cl.count);
+  for (int64_t j = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; j < n;
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = cl.rows[j];
+    const int rk = rank_of_row(rank_of, row, nB, R);
+    if (rk >= 0 && need[rk] > 0 && cl.keys[j] == prefix[rk]) atomicAdd(&tie_take[row], 1);
+  }
 }
 
 // rows in (head, query block) order take the ties each rank still needs. Ties are rare:
@@ -222,9 +297,15 @@ __global__ void __launch_bounds__(256) sasa_bits_kernel(const uint64_t* __restri
 
 }  // namespace
 
+// compact list capacity: a sixteenth of all entries (at least 256)
+static size_t sasa_compact_capacity(const Dims& D) {
+  const size_t c = (static_cast<size_t>(D.rows) * static_cast<size_t>(D.nB) + 15) / 16;
+  return c < 256 ? 256 : c;
+}
+
 size_t sasa_extra_bytes(const Dims& D) {
   return align_up(static_cast<size_t>(D.rows) * 4, 256) + align_up(kSasaMaxRanks * kSasaBins * 4, 256) +
-         4 * align_up(kSasaMaxRanks * 8, 256);
+         4 * align_up(kSasaMaxRanks * 8, 256) + align_up(8, 256) + align_up(sasa_compact_capacity(D) * 8, 256) * 2;
 }
 
 cudaError_t launch_sasa(const Dims& D, const double* pq, const double* pk, const int32_t* rank_of, int R,
@@ -241,11 +322,23 @@ cudaError_t launch_sasa(const Dims& D, const double* pq, const double* pk, const
   unsigned long long* pmask = reinterpret_cast<unsigned long long*>(extra + off);
   off += align_up(kSasaMaxRanks * 8, 256);
   long long* need = reinterpret_cast<long long*>(extra + off);
+  off += align_up(kSasaMaxRanks * 8, 256);
+  CompactList cl;
+  cl.count = reinterpret_cast<unsigned long long*>(extra + off);
+  off += align_up(8, 256);
+  cl.capacity = sasa_compact_capacity(D);
+  cl.keys = reinterpret_cast<uint64_t*>(extra + off);
+  off += align_up(cl.capacity * 8, 256);
+  cl.rows = reinterpret_cast<int64_t*>(extra + off);
+  CompactList full = cl;  // the same list, not used yet: passes read every entry
+  full.count = nullptr;
 
   const int nB = static_cast<int>(D.nB), nWords = static_cast<int>(D.nWords);
   const unsigned row_grid = static_cast<unsigned>((D.rows + 7) / 8);
   cudaError_t e = cudaMemsetAsync(hist, 0, kSasaMaxRanks * kSasaBins * 4, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(total, 0, kSasaMaxRanks * 8, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(cl.count, 0, 8, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(tie_take, 0, static_cast<size_t>(D.rows) * 4, st);
   // the block logits: exported by the routing pass (mask->logits), else recomputed
   const double* logits = m->logits;
   if (!logits && e == cudaSuccess) {
@@ -266,10 +359,14 @@ cudaError_t launch_sasa(const Dims& D, const double* pq, const double* pk, const
     if (e != cudaSuccess) return e;
   }
   for (int shift = 56; shift >= 0; shift -= 8) {
-    sasa_hist_kernel<<<148 * 4, 512, hist_smem, st>>>(keys, D.rows, nB, rank_of, R, prefix, pmask, need, shift, hist);
+    sasa_hist_kernel<<<148 * 4, 512, hist_smem, st>>>(keys, D.rows, nB, rank_of, R, prefix, pmask, need, shift, hist,
+                                                      shift < 48 ? cl : full);
     sasa_pick_kernel<<<1, kSasaMaxRanks, 0, st>>>(hist, R, shift, prefix, pmask, need, dev_status);
+    if (shift == 48)
+      sasa_compact_kernel<<<148 * 4, 512, 0, st>>>(keys, D.rows, nB, rank_of, R, prefix, pmask, need, cl);
   }
-  sasa_ties_count_kernel<<<row_grid, 256, 0, st>>>(keys, D.rows, nB, rank_of, R, prefix, need, tie_take);
+  sasa_ties_count_kernel<<<row_grid, 256, 0, st>>>(keys, D.rows, nB, rank_of, R, prefix, need, tie_take, cl);
+  sasa_ties_compact_kernel<<<148 * 4, 512, 0, st>>>(nB, rank_of, R, prefix, need, tie_take, cl);
   sasa_ties_alloc_kernel<<<1, 1024, 0, st>>>(D.rows, nB, rank_of, R, need, tie_take);
   sasa_bits_kernel<<<row_grid, 256, 0, st>>>(keys, D.rows, nB, nWords, rank_of, R, prefix, pmask, need, tie_take,
                                               ws.bits, ws.row_cnt);

@@ -76,7 +76,13 @@ def _check(wl, L, rank_of, budget, order=2, max_amb=None):
         order_row = O.routing_order(logits[h, a])
         if not amb[row]:
             assert new == set(order_row[: len(new)].tolist())
-    # tiles, costs and work list rebuilt consistently
+    _check_rebuilt(g1, BH, nB, order)
+    return run
+
+
+def _check_rebuilt(g1, BH, nB, order):
+    """tiles, costs and work list rebuilt consistently with the new CSR"""
+    rp, ci = g1["row_ptr"], g1["col_idx"]
     tiles = C.expected_tiles(rp, ci, BH, nB)
     costs = np.array([len(t) for t in tiles])
     np.testing.assert_array_equal(g1["tile_cost"], costs)
@@ -84,7 +90,6 @@ def _check(wl, L, rank_of, budget, order=2, max_amb=None):
     np.testing.assert_array_equal(g1["tile_col"], np.concatenate([np.array(t, dtype=np.int64) for t in tiles]))
     np.testing.assert_array_equal(g1["worklist"], C.expected_worklist(costs, BH, (nB + 1) // 2, order))
     np.testing.assert_array_equal(g1["head_kept"], [rp[(h + 1) * nB] - rp[h * nB] for h in range(BH)])
-    return run
 
 
 SMALL = [
@@ -156,3 +161,32 @@ def test_sasa_reads_logits_exported_by_routing(wid_or_wl):
         np.testing.assert_array_equal(g1[key], g1a[key])
     # the exported logits are read, not overwritten
     np.testing.assert_array_equal(lay.mask.logits.cpu().numpy(), got)
+
+
+@pytest.mark.parametrize("p,budget", [(0.9, [1000, 2500]), (0.95, [1000, 700])])
+def test_sasa_every_candidate_ties(p, budget):
+    """Q = 0, so every block logit is 0 and every skipped entry has the importance 1/nB,
+    exactly, on both sides: the whole budget is placed by the tie rule (rows in head, then
+    query block order; lower key block first). nB = 128 and 4 heads: routing keeps 116
+    blocks of every row at p = 0.9 and 122 at p = 0.95, so a tenth / a twentieth of all
+    entries are candidates, on either side of the compact list's capacity (a sixteenth of
+    the entries): the select runs over every entry in the first case and over the compact
+    list in the second, and both must place the budget exactly as the oracle does."""
+    import dataclasses
+    wl = synth.custom_workload(8, 32, 32, 4, 64, "bf16", seed=75, p=p, k_floor=1)
+    L = synth.make_layer(wl)
+    L = dataclasses.replace(L, q=np.zeros_like(L.q), q_bits=np.zeros_like(L.q_bits))
+    BH, nB = wl.B * wl.H, wl.nB
+    assert nB == 128
+    rank_of = [h % 2 for h in range(BH)]
+    run, g0, g1, added = _run_sasa(wl, L, rank_of, budget)
+    len0 = np.diff(g0["row_ptr"])
+    assert np.all(len0 == {0.9: 116, 0.95: 122}[p])
+    logits = np.zeros((BH, nB, nB))
+    want = S.augment(logits, len0, rank_of, budget)
+    np.testing.assert_array_equal(np.diff(g1["row_ptr"]), want)
+    np.testing.assert_array_equal(added, budget)
+    rp, ci = g1["row_ptr"], g1["col_idx"]
+    for row in range(BH * nB):  # equal logits: the routing order is the block order
+        np.testing.assert_array_equal(O.row_list(rp, ci, row), np.arange(want[row]))
+    _check_rebuilt(g1, BH, nB, 2)
