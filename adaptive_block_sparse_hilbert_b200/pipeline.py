@@ -90,11 +90,12 @@ def ramp_sizes(H: int, steady: int = 4):
 
 class HostPipelinedLayer:
     """One layer from page-locked host Q, K, V [B, N, H, d] to host O, pipelined over head
-    groups: one stream copies group g+1's head slices in while another runs group g's
-    reorder -> route -> attention -> inverse reorder and a third copies group g-1's output
-    back. Heads are independent along the whole path, so every group is an ordinary
-    SparseAttentionLayer on a shape with fewer heads, and the output equals the one-shot
-    layer's bit for bit.
+    groups: one stream copies group g+1's head slices in while the compute streams run
+    groups' reorder -> route -> attention -> inverse reorder and another stream copies group
+    g-1's output back. Groups alternate between two compute streams, so a group's launches
+    can start on the SMs that the previous group's attention tail leaves idle. Heads are
+    independent along the whole path, so every group is an ordinary SparseAttentionLayer on
+    a shape with fewer heads, and the output equals the one-shot layer's bit for bit.
 
     Consecutive forward() calls overlap too: a call's copy-in of a group waits only for the
     previous call's compute of that group (the last reader of the group's input buffers),
@@ -110,9 +111,10 @@ class HostPipelinedLayer:
 
     def __init__(self, shape: fva.fva_shape, p: float, k_floor: int, groups=None,
                  order: int = fva.FVA_ORDER_HEAD_LPT, device: str = "cuda", v_fp16: bool = True,
-                 curve: int = fva.FVA_CURVE_HILBERT, sizes=None):
+                 curve: int = fva.FVA_CURVE_HILBERT, sizes=None, compute_streams: int = 2):
         """groups: None for the ramp schedule (ramp_sizes), or a number of equal groups;
-        sizes: explicit head counts per group (overrides groups)."""
+        sizes: explicit head counts per group (overrides groups); compute_streams: streams
+        the groups' compute alternates between (1 runs the groups one after another)."""
         s = shape
         H = s.H
         if sizes is None and groups is None:
@@ -139,7 +141,7 @@ class HostPipelinedLayer:
             for lst in (self.q_in, self.k_in, self.v_in, self.o_out):
                 lst.append(torch.empty((s.B, self.N, n, s.d), dtype=dt, device=device))
         self.s_in = torch.cuda.Stream(device=device)
-        self.s_comp = torch.cuda.Stream(device=device)
+        self.s_comp = [torch.cuda.Stream(device=device) for _ in range(max(1, int(compute_streams)))]
         self.s_out = torch.cuda.Stream(device=device)
         G = len(self.heads)
         self.in_ready = [torch.cuda.Event() for _ in range(G)]    # group's inputs on the device
@@ -149,8 +151,11 @@ class HostPipelinedLayer:
         # the buffers (and each group's token order) were made on the current stream
         made = torch.cuda.Event()
         made.record(torch.cuda.current_stream())
-        for st in (self.s_in, self.s_comp, self.s_out):
+        for st in self._streams():
             st.wait_event(made)
+
+    def _streams(self):
+        return [self.s_in, *self.s_comp, self.s_out]
 
     def forward(self, q_host, k_host, v_host, o_host):
         """Enqueue one layer and return the stream that copies its output out (see the
@@ -166,11 +171,12 @@ class HostPipelinedLayer:
                 fva.fva_copy_strided(dst, width, src[:, :, h0:h0 + n, :], row, width, rows, self.s_in)
             self.in_ready[g].record(self.s_in)
         for g, ((h0, n), layer) in enumerate(zip(self.heads, self.layers)):
-            self.s_comp.wait_event(self.in_ready[g])
+            st = self.s_comp[g % len(self.s_comp)]
+            st.wait_event(self.in_ready[g])
             if self.started:
-                self.s_comp.wait_event(self.out_done[g])
-            layer.forward(self.q_in[g], self.k_in[g], self.v_in[g], self.o_out[g], self.s_comp)
-            self.comp_done[g].record(self.s_comp)
+                st.wait_event(self.out_done[g])
+            layer.forward(self.q_in[g], self.k_in[g], self.v_in[g], self.o_out[g], st)
+            self.comp_done[g].record(st)
             self.s_out.wait_event(self.comp_done[g])
             width = n * s.d * self.esize
             fva.fva_copy_strided(o_host[:, :, h0:h0 + n, :], row, self.o_out[g], width, width, rows, self.s_out)
@@ -182,16 +188,15 @@ class HostPipelinedLayer:
         """Make the layer's streams wait for the work already enqueued on `stream` (default:
         the current stream), e.g. a timing event or a producer of the host inputs."""
         st = torch.cuda.current_stream() if stream is None else stream
-        for side in (self.s_in, self.s_comp, self.s_out):
+        for side in self._streams():
             side.wait_stream(st)
 
     def wait(self, stream=None):
         """Make `stream` (default: the current stream) wait until every enqueued forward()
         has finished, its output copied to host memory."""
         st = torch.cuda.current_stream() if stream is None else stream
-        st.wait_stream(self.s_in)
-        st.wait_stream(self.s_comp)
-        st.wait_stream(self.s_out)
+        for side in self._streams():
+            st.wait_stream(side)
 
     def dev_status(self):
         """Largest device error code any group reported (0 = none)."""

@@ -999,7 +999,7 @@ def run_gpu(args):
                     "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h),
                     "how": f"pipelined over head groups of {e2e_sizes} heads (copy in / compute / copy out "
-                           f"on three streams; consecutive layers overlap), {n_e2e} layers timed",
+                           f"on four streams, two of them computing; consecutive layers overlap), {n_e2e} layers timed",
                     "serial_ms": round(whole_job_ms_per_layer(e2e_serial_ms, world), 3),
                     "single_layer_ms": round(e2e_single_ms, 3)},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,

@@ -1,5 +1,6 @@
-"""The host-pipelined layer (head groups copied in, computed and copied out on three
-streams) writes the same output as the one-shot device layer, bit for bit."""
+"""The host-pipelined layer (head groups copied in, computed on two alternating compute
+streams, or one, and copied out) writes the same output as the one-shot device layer, bit
+for bit."""
 import numpy as np
 import pytest
 
@@ -9,8 +10,9 @@ from tests import _common as C
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("B,H,groups", [(1, 5, 3), (1, 4, 4), (1, 6, 1), (1, 7, None), (2, 5, 2)])
-def test_pipelined_equals_one_shot(B, H, groups):
+@pytest.mark.parametrize("B,H,groups,streams", [(1, 5, 3, 2), (1, 4, 4, 2), (1, 6, 1, 2), (1, 7, None, 2),
+                                                (2, 5, 2, 2), (1, 5, 3, 1), (1, 7, None, 3)])
+def test_pipelined_equals_one_shot(B, H, groups, streams):
     import torch
     from adaptive_block_sparse_hilbert_b200 import fva, pipeline
     wl = synth.custom_workload(3, 10, 13, H, 128, "bf16", seed=81, B=B)
@@ -22,7 +24,7 @@ def test_pipelined_equals_one_shot(B, H, groups):
     one.forward(q, k, v, o_ref)
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
     oh = torch.zeros_like(qh).pin_memory()
-    pipe = pipeline.HostPipelinedLayer(s, wl.p, wl.k_floor, groups=groups)
+    pipe = pipeline.HostPipelinedLayer(s, wl.p, wl.k_floor, groups=groups, compute_streams=streams)
     pipe.forward(qh, kh, vh, oh)
     torch.cuda.synchronize()
     assert pipe.dev_status() == 0 and int(one.dev_status.item()) == 0
