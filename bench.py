@@ -413,6 +413,34 @@ def fp64_gemm_peak_tflops(dev, n: int = 8192, reps: int = 5) -> float:
     return 2.0 * n ** 3 / (best * 1e-3) / 1e12
 
 
+def library_dense_report(layer, dense_flops: float, dense_ms: float, stream):
+    """Context for the dense kernel: the vendor's fused attention (torch SDPA restricted to
+    its cuDNN backend) on the same Hilbert-ordered Q, K and a bf16 copy of V, [B, H, N, d],
+    timed the same way. A measurement of the machine, outside the path."""
+    import torch
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    try:
+        v = layer.vh.to(torch.bfloat16)
+        with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+            for _ in range(2):
+                torch.nn.functional.scaled_dot_product_attention(layer.qh, layer.kh, v)
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            for _ in range(3):
+                torch.nn.functional.scaled_dot_product_attention(layer.qh, layer.kh, v)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / 3
+        del v
+        torch.cuda.empty_cache()
+    except Exception as e:  # no cuDNN attention for this shape or build
+        return {"what": "torch SDPA, cuDNN backend", "error": str(e)[:160]}
+    return {"what": "torch SDPA restricted to the cuDNN backend (vendor fused attention, dense, bf16), same inputs",
+            "ms": round(ms, 3), "tflops": round(dense_flops / (ms * 1e-3) / 1e12, 1),
+            "fva_dense_ms_over_library_ms": round(dense_ms / ms, 3)}
+
+
 def imbalance(costs: np.ndarray, BH: int, n_pairs: int, slots: int):
     out = {}
     ids = np.arange(costs.size)
@@ -781,6 +809,7 @@ def run_gpu(args):
 
     # dense density-1 reference kernel (same launch family), timed separately
     dense_ms = None
+    dense_library = None
     if not args.no_dense:
         od = torch.empty_like(layer.qh)
         for _ in range(2):
@@ -793,6 +822,7 @@ def run_gpu(args):
         torch.cuda.synchronize()
         dense_ms = e0.elapsed_time(e1) / 3
         del od
+        dense_library = library_dense_report(layer, dense_flops, dense_ms, stream)
 
     # one traced attention launch (outside the timed region): measured SM-level balance
     sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -968,6 +998,7 @@ def run_gpu(args):
             "density_per_head": [round(float(x) / (nB * nB), 4) for x in per_step[0][3]],
             "dense_attn_ms": round(dense_ms, 3) if dense_ms else None,
             "dense_attn_tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 1) if dense_ms else None,
+            "dense_library": dense_library,
             "reorder_gbs": round(reorder_bytes / (t_reorder * 1e-3) / 1e9, 1),
             "reorder_hbm_frac": round(reorder_bytes / (t_reorder * 1e-3) / 1e9 / hbm, 4),
             "route": {"gbs": round(route_bytes / (t_route * 1e-3) / 1e9, 1),
