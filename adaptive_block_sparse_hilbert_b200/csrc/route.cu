@@ -149,7 +149,7 @@ constexpr double kFix = 4503599627370496.0;     // 2^52: fixed-point unit of imp
 struct WarpArena {
   double* s;          // [nB] the row's logits
   uint64_t* hw;       // [kNBK] bucket mass (fixed point); last: masses of the final candidates
-  int32_t* list;      // [nB] candidate block indices
+  uint16_t* list;     // [nB] candidate block indices (routable nB < 2^16)
   int32_t* hcnt;      // [kNBK] bucket counts
   uint32_t* words;    // [nWords] kept bitmask of the row
 };
@@ -158,7 +158,7 @@ __host__ __device__ inline size_t warp_arena_bytes(int nB, int nWords) {
   size_t b = 0;
   b += align_up(static_cast<size_t>(nB) * 8, 16);
   b += kNBK * 8;
-  b += align_up(static_cast<size_t>(nB) * 4, 16);
+  b += align_up(static_cast<size_t>(nB) * 2, 16);
   b += kNBK * 4;
   b += align_up(static_cast<size_t>(nWords) * 4, 16);
   return b;
@@ -171,8 +171,8 @@ __device__ inline WarpArena make_arena(uint8_t* base, int nB, int nWords) {
   off += align_up(static_cast<size_t>(nB) * 8, 16);
   A.hw = reinterpret_cast<uint64_t*>(base + off);
   off += kNBK * 8;
-  A.list = reinterpret_cast<int32_t*>(base + off);
-  off += align_up(static_cast<size_t>(nB) * 4, 16);
+  A.list = reinterpret_cast<uint16_t*>(base + off);
+  off += align_up(static_cast<size_t>(nB) * 2, 16);
   A.hcnt = reinterpret_cast<int32_t*>(base + off);
   off += kNBK * 4;
   A.words = reinterpret_cast<uint32_t*>(base + off);
@@ -305,7 +305,7 @@ __device__ Pivot select_pivot(const WarpArena& A, int nB, double smax, double sm
       const unsigned m = __ballot_sync(0xffffffffu, in);
       __syncwarp();
       if (in) {
-        A.list[newc + __popc(m & ((1u << lane) - 1u))] = b;
+        A.list[newc + __popc(m & ((1u << lane) - 1u))] = static_cast<uint16_t>(b);
         nlo = fmin(nlo, s);
         nhi = fmax(nhi, s);
       }
@@ -318,7 +318,7 @@ __device__ Pivot select_pivot(const WarpArena& A, int nB, double smax, double sm
     hi = warp_max_d(nhi);
   }
   if (implicit) {
-    for (int i = lane; i < c; i += 32) A.list[i] = i;
+    for (int i = lane; i < c; i += 32) A.list[i] = static_cast<uint16_t>(i);
     __syncwarp();
   }
   // masses of the remaining candidates, kept in the bucket array when they fit (the

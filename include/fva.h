@@ -86,7 +86,7 @@ enum {
  *   Hg, Wg <= 65536; N = T*Hg*Wg <= 2^31 - 1; nB <= 524280; B*H <= 65535;
  *   B*H*nB <= 2^31 - 1;
  *   d * sizeof(dtype) in {64, 128, 256, 512, 1024} bytes;
- *   routing (fva_route, fva_route_noalloc, fva_sasa_augment): nB <= 9458, the largest
+ *   routing (fva_route, fva_route_noalloc, fva_sasa_augment): nB <= 11326, the largest
  *   count for which two rows' float64 working sets fit one CTA's 227 KB of shared
  *   memory, and B*H*nB*nB <= 2^31 - 1 (int32 CSR offsets);
  *   attention: see fva_sparse_attn. */

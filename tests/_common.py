@@ -168,10 +168,10 @@ def default_scale(d):
 
 
 def largest_routable_workload():
-    """One head at the routing kernel's largest block count: 778 x 778 = 605,284 tokens,
-    nB = 9458 (a ragged tail of 36), d = 64. Heads drawn with tau in logU(2, 2.5) give a
-    density near 0.18 with row lengths from a few dozen to thousands of blocks."""
-    return synth.custom_workload(1, 778, 778, 1, 64, "bf16", seed=41, tau=("logU", 2.0, 2.5))
+    """One head at the routing kernel's largest block count: 837 x 866 = 724,842 tokens,
+    nB = 11326 (a ragged tail of 42), d = 64. Heads drawn with tau in logU(2, 2.5) give a
+    low density with row lengths from a few dozen to thousands of blocks."""
+    return synth.custom_workload(1, 837, 866, 1, 64, "bf16", seed=41, tau=("logU", 2.0, 2.5))
 
 
 def sampled_attention_errors(run, wl, L, g, n_per_head, seed, curve=0):

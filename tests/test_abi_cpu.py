@@ -70,12 +70,12 @@ def test_invalid_shapes_rejected():
 
 def test_routing_limit_on_block_count():
     """Routing keeps two rows' float64 working sets in one CTA's shared memory, which
-    bounds nB at 9458; one block more is rejected on the host before any launch."""
+    bounds nB at 11326; one block more is rejected on the host before any launch."""
     P = ctypes.c_void_p
     one = P(16)  # non-null dummy pointer; every call below fails validation first
-    ok = fva.make_shape(1, 1, 64, 1, 778, 778)        # N = 605,284: nB = 9458
-    over = fva.make_shape(1, 1, 64, 10, 1, 60532)     # N = 605,320: nB = 9459
-    assert fva.fva_num_blocks(ok) == 9458 and fva.fva_num_blocks(over) == 9459
+    ok = fva.make_shape(1, 1, 64, 1, 837, 866)        # N = 724,842: nB = 11326
+    over = fva.make_shape(1, 1, 64, 1, 840, 863)      # N = 724,920: nB = 11327
+    assert fva.fva_num_blocks(ok) == 11326 and fva.fva_num_blocks(over) == 11327
     assert fva.fva_route_workspace_bytes(ok, 0) > 0 and fva.fva_route_workspace_bytes(ok, 1) > 0
     assert fva.fva_sasa_workspace_bytes(ok) > 0
     assert fva.fva_route_workspace_bytes(over, 0) == 0 and fva.fva_route_workspace_bytes(over, 1) == 0

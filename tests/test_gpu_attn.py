@@ -182,7 +182,7 @@ def test_sparse_full_size_sampled(wid):
 
 
 def test_sparse_at_largest_routable_shape():
-    """One head of 605,284 tokens (nB = 9458, the routing limit), 4,729 pair tiles."""
+    """One head of 724,842 tokens (nB = 11326, the routing limit), 5,663 pair tiles."""
     wl = C.largest_routable_workload()
     _sampled_check(wl, synth.make_layer(wl), 10, 41)
 

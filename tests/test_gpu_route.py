@@ -144,11 +144,11 @@ def test_route_and_attend_720p_p_sweep(p):
 
 
 def test_route_at_largest_routable_shape():
-    """nB = 9458, the largest block count routing supports (one more is rejected on the
+    """nB = 11326, the largest block count routing supports (one more is rejected on the
     host before any launch; see test_abi_cpu.py). The selection kernel runs with its
     largest per-row shared-memory arena here."""
     wl = C.largest_routable_workload()
-    assert wl.nB == 9458 and wl.N % 64 == 36
+    assert wl.nB == 11326 and wl.N % 64 == 42
     # at this nB the entry at a row's cut holds ~1e-4 of the row's mass, so the oracle's
     # 1e-6 ambiguity band covers a few percent of the rows; mismatches outside the band
     # must still be zero
