@@ -658,13 +658,17 @@ __global__ void __launch_bounds__(256) emit_kernel(const uint32_t* __restrict__ 
 // ---------------------------------------------------------------------------------
 // Tiles from a caller-made CSR
 // ---------------------------------------------------------------------------------
+// One warp per row: the row's bitmask is built in shared memory (nWords words per warp),
+// then written out in whole words.
 __global__ void __launch_bounds__(256) csr_to_bits_kernel(const int32_t* __restrict__ row_ptr,
                                                           const int32_t* __restrict__ col_idx, int64_t rows,
                                                           int nB, int nWords, uint32_t* bits, int32_t* dev_status) {
+  extern __shared__ uint32_t row_words[];  // [8][nWords]
   const int lane = threadIdx.x & 31;
   const int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= rows) return;
-  for (int k = lane; k < nWords; k += 32) bits[r * nWords + k] = 0u;
+  uint32_t* w = row_words + (threadIdx.x >> 5) * nWords;
+  for (int k = lane; k < nWords; k += 32) w[k] = 0u;
   __syncwarp();
   const int32_t lo = row_ptr[r], hi = row_ptr[r + 1];
   for (int32_t i = lo + lane; i < hi; i += 32) {
@@ -673,8 +677,10 @@ __global__ void __launch_bounds__(256) csr_to_bits_kernel(const int32_t* __restr
       report(dev_status, FVA_DEVERR_BAD_LIST);
       continue;
     }
-    atomicOr(&bits[r * nWords + (c >> 5)], 1u << (c & 31));
+    atomicOr(&w[c >> 5], 1u << (c & 31));
   }
+  __syncwarp();
+  for (int k = lane; k < nWords; k += 32) bits[r * nWords + k] = w[k];
 }
 
 __global__ void __launch_bounds__(256) tile_cost_kernel(const uint32_t* __restrict__ bits, int nB, int nWords,
@@ -779,7 +785,13 @@ cudaError_t launch_route_scores(const Dims& D, const double* pq, const double* p
 
 cudaError_t launch_csr_to_bits(const Dims& D, const fva_mask* m, uint32_t* bits, int32_t* dev_status,
                                cudaStream_t st) {
-  csr_to_bits_kernel<<<static_cast<int>((D.rows + 7) / 8), 256, 0, st>>>(
+  const size_t smem = static_cast<size_t>(D.nWords) * 4 * 8;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(csr_to_bits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  csr_to_bits_kernel<<<static_cast<int>((D.rows + 7) / 8), 256, smem, st>>>(
       m->row_ptr, m->col_idx, D.rows, static_cast<int>(D.nB), static_cast<int>(D.nWords), bits, dev_status);
   return cudaGetLastError();
 }

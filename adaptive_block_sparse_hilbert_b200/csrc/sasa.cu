@@ -41,10 +41,12 @@ __device__ __forceinline__ int rank_of_row(const int32_t* rank_of, int64_t row, 
 
 // per row: row maximum, Z = sum exp(s - max), then one key per entry; counts candidates.
 // `logits` and `keys_out` may be the same array (the keys then replace the logits: every
-// lane writes only the entries it has just read, after the row's reductions).
+// lane writes only the entries it has just read, after the row's reductions). Rows of a
+// rank without a budget are left alone: no later pass reads their keys.
 __global__ void __launch_bounds__(256) sasa_keys_kernel(const double* logits, uint64_t* keys_out,
                                                         const uint32_t* __restrict__ bits, int64_t rows, int nB,
                                                         int nWords, const int32_t* __restrict__ rank_of, int R,
+                                                        const int64_t* __restrict__ budget,
                                                         unsigned long long* total, int32_t* dev_status) {
   const int lane = threadIdx.x & 31;
   const int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -52,6 +54,7 @@ __global__ void __launch_bounds__(256) sasa_keys_kernel(const double* logits, ui
   const double* s = logits + r * nB;
   const int rk = rank_of_row(rank_of, r, nB, R);
   if (rk < 0 && lane == 0 && (r % nB) == 0) report(dev_status, FVA_DEVERR_BAD_LIST);
+  if (rk >= 0 && budget[rk] <= 0) return;
   double mx = -INFINITY;
   for (int b = lane; b < nB; b += 32) mx = fmax(mx, s[b]);
   mx = warp_max_d(mx);
@@ -168,29 +171,59 @@ __global__ void __launch_bounds__(512) sasa_hist_kernel(const uint64_t* __restri
     if (sh[i]) atomicAdd(&hist[i], sh[i]);
 }
 
-// one thread per rank: the digit where the count from the top reaches `need`
-__global__ void sasa_pick_kernel(unsigned* hist, int R, int shift, unsigned long long* prefix,
-                                 unsigned long long* pmask, long long* need, int32_t* dev_status) {
-  const int r = threadIdx.x;
+// one warp per rank: the digit where the count from the top reaches `need`. Lane l holds
+// bins 8l .. 8l+7; a suffix sum over the lanes above gives each lane the count of the
+// digits above its bins, and the lane whose bins hold the crossing picks it.
+__global__ void __launch_bounds__(32) sasa_pick_kernel(unsigned* hist, int R, int shift, unsigned long long* prefix,
+                                                       unsigned long long* pmask, long long* need,
+                                                       int32_t* dev_status) {
+  const int r = blockIdx.x;
+  const int lane = threadIdx.x;
   if (r >= R) return;
   unsigned* h = hist + r * kSasaBins;
-  if (need[r] > 0) {
-    long long above = 0;
-    int d = kSasaBins - 1;
-    for (; d >= 0; --d) {
-      if (above + h[d] >= need[r]) break;
-      above += h[d];
+  unsigned c[8];
+  long long mine = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    c[q] = h[8 * lane + q];
+    mine += c[q];
+  }
+  const long long nd = need[r];
+  if (nd > 0) {
+    long long above = mine;  // inclusive suffix sum: bins 8 lane .. 255
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long t = __shfl_down_sync(0xffffffffu, above, o);
+      if (lane + o < 32) above += t;
     }
-    if (d < 0) {  // fewer matching entries than needed: cannot happen when counts are right
-      report(dev_status, FVA_DEVERR_MASK);
-      need[r] = 0;
-    } else {
+    above -= mine;  // bins above this lane's eight
+    int d = -1;
+    long long before = 0;
+    if (above < nd && above + mine >= nd) {
+      long long run = above;
+      for (int q = 7; q >= 0; --q) {
+        if (run + c[q] >= nd) {
+          d = 8 * lane + q;
+          before = run;
+          break;
+        }
+        run += c[q];
+      }
+    }
+    const unsigned who = __ballot_sync(0xffffffffu, d >= 0);
+    if (who == 0) {  // fewer matching entries than needed: cannot happen when counts are right
+      if (lane == 0) {
+        report(dev_status, FVA_DEVERR_MASK);
+        need[r] = 0;
+      }
+    } else if (lane == __ffs(who) - 1) {
       prefix[r] |= static_cast<unsigned long long>(d) << shift;
       pmask[r] |= 255ull << shift;
-      need[r] -= above;
+      need[r] = nd - before;
     }
   }
-  for (int i = 0; i < kSasaBins; ++i) h[i] = 0u;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) h[8 * lane + q] = 0u;
 }
 
 // entries equal to tau_r per row (tie candidates)
@@ -240,12 +273,11 @@ __global__ void __launch_bounds__(1024) sasa_ties_alloc_kernel(int64_t rows, int
   __shared__ int has[1024];
   __shared__ long long left[kSasaMaxRanks];
   const int64_t chunk = (rows + blockDim.x - 1) / blockDim.x;
-  const int64_t lo = threadIdx.x * chunk;
-  const int64_t hi = lo + chunk < rows ? lo + chunk : rows;
-  int any = 0;
-  for (int64_t row = lo; row < hi; ++row) any |= tie_take[row] != 0;
-  has[threadIdx.x] = any;
+  has[threadIdx.x] = 0;
   if (threadIdx.x < R) left[threadIdx.x] = need[threadIdx.x] > 0 ? need[threadIdx.x] : 0;
+  __syncthreads();
+  for (int64_t row = threadIdx.x; row < rows; row += blockDim.x)  // coalesced
+    if (tie_take[row] != 0) has[row / chunk] = 1;
   __syncthreads();
   if (threadIdx.x != 0) return;
   for (int c = 0; c < static_cast<int>(blockDim.x); ++c) {
@@ -277,6 +309,14 @@ __global__ void __launch_bounds__(256) sasa_bits_kernel(const uint64_t* __restri
   const int rk = rank_of_row(rank_of, r, nB, R);
   const bool all = rk >= 0 && need[rk] < 0;
   const bool thr = rk >= 0 && pmask[rk] != 0;
+  if (!all && !thr) {  // nothing added to this row: count its kept blocks, keys unread
+    int kept = 0;
+    for (int k = lane; k < nWords; k += 32) kept += __popc(bits[r * nWords + k]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, o);
+    if (lane == 0) row_cnt[r] = kept;
+    return;
+  }
   const uint64_t tau = thr ? prefix[rk] : ~0ull;
   const int ties = tie_take[r];
   int tie_seen = 0, kept = 0;
@@ -348,7 +388,7 @@ cudaError_t launch_sasa(const Dims& D, const double* pq, const double* pk, const
   if (e == cudaSuccess) e = launch_csr_to_bits(D, m, ws.bits, dev_status, st);
   if (e != cudaSuccess) return e;
   sasa_keys_kernel<<<row_grid, 256, 0, st>>>(logits, reinterpret_cast<uint64_t*>(ws.scores), ws.bits, D.rows, nB,
-                                             nWords, rank_of, R, total, dev_status);
+                                             nWords, rank_of, R, budget, total, dev_status);
   sasa_init_kernel<<<1, kSasaMaxRanks, 0, st>>>(budget, R, total, prefix, pmask, need, added);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -361,7 +401,7 @@ cudaError_t launch_sasa(const Dims& D, const double* pq, const double* pk, const
   for (int shift = 56; shift >= 0; shift -= 8) {
     sasa_hist_kernel<<<148 * 4, 512, hist_smem, st>>>(keys, D.rows, nB, rank_of, R, prefix, pmask, need, shift, hist,
                                                       shift < 48 ? cl : full);
-    sasa_pick_kernel<<<1, kSasaMaxRanks, 0, st>>>(hist, R, shift, prefix, pmask, need, dev_status);
+    sasa_pick_kernel<<<R, 32, 0, st>>>(hist, R, shift, prefix, pmask, need, dev_status);
     if (shift == 48)
       sasa_compact_kernel<<<148 * 4, 512, 0, st>>>(keys, D.rows, nB, rank_of, R, prefix, pmask, need, cl);
   }
