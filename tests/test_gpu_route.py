@@ -74,6 +74,18 @@ def test_route_small(wl, p, kf, order):
     _check_route(wl, L, p, kf, order)
 
 
+@pytest.mark.parametrize("wl", [
+    synth.custom_workload(3, 16, 21, 3, 32, "bf16", seed=28),   # d = 32: the logit GEMM runs two d-chunks
+    synth.custom_workload(3, 16, 21, 2, 16, "f32", seed=29),    # d = 16: one d-chunk
+    synth.custom_workload(2, 12, 15, 2, 256, "bf16", seed=30),  # d = 256: sixteen d-chunks through the ring
+], ids=lambda w: w.name)
+def test_route_other_head_dims(wl):
+    """Routing at the head dimensions the attention kernel does not take (pooling, logits and
+    selection only): the block-logit GEMM stages d in chunks of 16 through a three-stage
+    ring, so d = 16, 32 and 256 cover one, two and many chunks."""
+    _check_route(wl, synth.make_layer(wl), wl.p, wl.k_floor, order=2)
+
+
 def test_route_internal_pooling_matches():
     wl = synth.custom_workload(3, 10, 13, 3, 64, "bf16", seed=25)
     L = synth.make_layer(wl)
