@@ -110,6 +110,17 @@ def test_sasa_small(wl, case):
     _check(wl, synth.make_layer(wl), rank_of, budget, order=[0, 1, 2, 2][["some", "all", "none", "one"].index(case)])
 
 
+def test_sasa_sixty_four_ranks():
+    """FVA_SASA_MAX_RANKS ranks, one head each (64 KB of per-CTA histograms, 64 digit
+    pickers), with budgets from none to more than a rank's skipped entries."""
+    wl = synth.custom_workload(3, 16, 20, 64, 64, "bf16", seed=76)
+    BH = wl.B * wl.H
+    rank_of = list(range(BH))
+    rng = np.random.default_rng(5)
+    budget = [int(x) for x in rng.choice([0, 1, 3, 17, 60, 10 ** 6], size=BH)]
+    _check(wl, synth.make_layer(wl), rank_of, budget)
+
+
 def test_sasa_720p_eight_ranks():
     wl = synth.WORKLOADS[2]
     BH = wl.B * wl.H
