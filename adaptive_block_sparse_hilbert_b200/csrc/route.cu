@@ -732,7 +732,9 @@ static cudaError_t launch_order_and_emit(const Dims& D, const fva_mask* m, int o
     order_lpt_kernel<<<static_cast<int>((D.tiles + 255) / 256), 256, 0, st>>>(m->tile_cost, D.tiles, m->worklist);
   } else {
     const size_t smem = static_cast<size_t>(D.nPairs) * 4;
-    cudaFuncSetAttribute(order_head_lpt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    const cudaError_t ea = cudaFuncSetAttribute(order_head_lpt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                static_cast<int>(smem));
+    if (ea != cudaSuccess) return ea;
     order_head_lpt_kernel<<<static_cast<int>(D.BH), 256, smem, st>>>(m->tile_cost, ws.head_load,
                                                                      static_cast<int>(D.BH),
                                                                      static_cast<int>(D.nPairs), m->worklist);
@@ -755,7 +757,9 @@ cudaError_t launch_route(const Dims& D, const double* pq, const double* pk, doub
   {
     const int rpc = select_rows_per_cta(D);
     const size_t smem = warp_arena_bytes(nB, static_cast<int>(D.nWords)) * rpc;
-    cudaFuncSetAttribute(route_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    const cudaError_t ea = cudaFuncSetAttribute(route_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                static_cast<int>(smem));
+    if (ea != cudaSuccess) return ea;
     const dim3 grid((nB + rpc - 1) / rpc, static_cast<unsigned>(D.BH));
     route_select_kernel<<<grid, 32 * rpc, smem, st>>>(ws.scores, nB, static_cast<int>(D.nWords),
                                                      static_cast<int>(D.nPairs), p, k_floor, ws.bits, ws.row_cnt,
