@@ -144,8 +144,10 @@ constexpr int kMaxLevels = 12;
 constexpr double kFix = 4503599627370496.0;     // 2^52: fixed-point unit of importance
 
 // Shared memory of one row's warp. The importances exp(s - max) are recomputed where they
-// are needed rather than kept (the same operation on the same inputs, so the same bits):
-// an fp64 copy of them would double the arena and halve the warps that fit on an SM.
+// are needed rather than kept (the same operation on the same inputs, so the same bits): an
+// fp64 copy of them beside the logits would nearly double the arena and cut the rows that fit
+// on an SM, and kept in place of the logits (which the passes then read again from L2) they
+// made the kernel slower. Candidates are 16-bit block indices for the same reason.
 struct WarpArena {
   double* s;          // [nB] the row's logits
   uint64_t* hw;       // [kNBK] bucket mass (fixed point); last: masses of the final candidates
